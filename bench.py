@@ -1,0 +1,327 @@
+"""Benchmark of one Wan DiT denoising-step forward on B200 (sm_100a).
+
+Default workload: Wan2.1-1.3B shapes at 480p, 81 frames -> latent
+[2,16,21,60,104] (L = 32760 tokens, 30 blocks), CFG batch 2 (one latent, two
+independent 226x4096 text contexts), random-init bf16 weights, timesteps
+cycling through {999, 500, 20}.  A step is one wan_dit_forward (the whole hot
+path).  `value` is whole-job tokens/s with inputs resident in HBM; `e2e` is the
+same metric through the C ABI with host buffers (copies inside the timed
+region).  Under torchrun every rank runs an independent replica (the forward
+does not shard), timing is max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+`--impl reference` times the float64 CPU oracle on a bounded sample of the
+same workload (see cpu_sample()).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/denoise-step & tokens/s, Wan-1.3B-shape 480p; % of B200 bf16 TC peak"
+DEFAULT_WORKLOAD = "wan1.3b-81f-480x832-cfg2"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def cpu_sample(w, rows_small=128, rows_big=384, seed=0):
+    """Time the float64 oracle on a bounded sample of the workload and scale it
+    to one full denoising step.
+
+    Sample: one block of the model (sample 0 of the batch) through the
+    oracle's row mode at two query-row counts R1 < R2 (keys/values over all L
+    tokens).  t(R) = a + b R fits the two timings; one full block is a + b L,
+    one step is B * N * (a + b L).  Returns (tokens/s, seconds per step, description)."""
+    import torch
+    from oracle import wan_oracle as O
+    from video_diffusion_transformer_dit_b200 import synth
+    cfg = dict(w["cfg"])
+    B, Cc, F, Hz, Wz = w["latent"]
+    L = O.token_count(F, Hz, Wz)
+    cfg1 = dict(cfg, num_blocks=1)
+    W = {k: v.double() for k, v in synth.make_weights(cfg1, seed=seed).items()}
+    lat = synth.make_latent((1, Cc, F, Hz, Wz), seed=seed).double()
+    ctx = synth.make_context(1, w["text_len"], cfg["text_dim"], seed=seed).double()
+    t = torch.full((1,), 999.0, dtype=torch.float64)
+    times = []
+    for R in (rows_small, rows_big):
+        rows = torch.linspace(0, L - 1, R).long()
+        t0 = time.perf_counter()
+        O.forward(lat, t, ctx, W, cfg1, rows=rows)
+        times.append(time.perf_counter() - t0)
+    b = max(0.0, (times[1] - times[0]) / (rows_big - rows_small))
+    a = max(0.0, times[0] - b * rows_small)
+    block_s = a + b * L
+    step_s = B * cfg["num_blocks"] * block_s
+    desc = (f"oracle row mode, 1 block x 1 sample at R={rows_small},{rows_big} query rows "
+            f"({times[0]:.1f}s, {times[1]:.1f}s); step = B*N*(a+b*L), extrapolated")
+    return B * L / step_s, step_s, desc, sum(times)
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from oracle import wan_oracle as O  # noqa: F401  (token law only used via configs)
+    from video_diffusion_transformer_dit_b200 import build, configs, synth
+    from video_diffusion_transformer_dit_b200.binding import WAN_OPT_KERNEL_TIMING, WanDiT
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = configs.workload(args.workload)
+    cfg = w["cfg"]
+    B, Cc, F, Hz, Wz = w["latent"]
+    L = F * (Hz // 2) * (Wz // 2)
+    Lc = w["text_len"]
+    peaks = load_peaks()
+
+    # random-init weights of the named shapes, generated on the device
+    W = synth.make_weights(cfg, seed=args.seed, device=str(dev))
+    lat = synth.make_latent(w["latent"], seed=args.seed, device=str(dev), same_across_batch=w.get("same_latent", False))
+    ctx = synth.make_context(B, Lc, cfg["text_dim"], seed=args.seed, device=str(dev))
+    if w["timesteps"] == "per_token":
+        ts = [synth.make_timestep_per_token(B, L, (Hz // 2) * (Wz // 2), seed=args.seed).to(dev)]
+    else:
+        ts = [synth.make_timestep(B, v).to(dev) for v in w["timesteps"]]
+    dit = WanDiT(cfg, max_batch=B, max_tokens=L, max_text=Lc, device=local_rank)
+    dit.load_weights(W)
+    del W
+    torch.cuda.synchronize()
+    vel = torch.empty(B, cfg["out_ch"], F, Hz, Wz, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(k):
+        dit.forward(lat, ts[k % len(ts)], ctx, velocity=vel)
+
+    for k in range(args.warmup):
+        step(k)
+    dit.sync()
+
+    dit.set_option(WAN_OPT_KERNEL_TIMING, 1)
+    step(0)                      # capture the timed graph outside the timed region
+    dit.sync()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(args.steps):
+        step(k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dit.sync()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    kt = {c: dit.kernel_time(c) for c in ("self_attention", "gemm", "cross_attention", "layernorm",
+                                         "rmsnorm_rope", "patchify", "embedding")}
+    launches = dit.last_launch_count()
+    dit.set_option(WAN_OPT_KERNEL_TIMING, 0)
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    lat_h = lat.cpu().pin_memory()
+    ctx_h = ctx.cpu().pin_memory()
+    ts_h = [t.cpu().pin_memory() for t in ts]
+    vel_h = torch.empty(vel.shape, dtype=torch.float32).pin_memory()
+    for k in range(2):
+        dit.forward(lat_h, ts_h[k % len(ts_h)], ctx_h, velocity=vel_h)
+    dit.sync()
+    if world > 1:
+        dist.barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    e2e_steps = max(1, min(args.steps, 3))
+    for k in range(e2e_steps):
+        dit.forward(lat_h, ts_h[k % len(ts_h)], ctx_h, velocity=vel_h)
+    e3.record(stream)
+    dit.sync()
+    ms_e2e = e2.elapsed_time(e3) / e2e_steps
+    h2d = lat_h.numel() * lat_h.element_size() + ctx_h.numel() * ctx_h.element_size() + \
+        ts_h[0].numel() * ts_h[0].element_size()
+    d2h = vel_h.numel() * vel_h.element_size()
+
+    if world > 1:
+        t = torch.tensor([ms, ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = t.tolist()
+
+    flops = dit.flops(B, F, Hz, Wz, Lc, int(w["timesteps"] == "per_token"))
+    # dominant kernel: self-attention, 4 * L^2 * head_dim * heads * B flops per launch
+    sa_ms, sa_n = kt["self_attention"]
+    sa_flops = 4.0 * L * L * cfg["dim"] * B
+    sa_avg_ms = sa_ms / max(1, sa_n)
+    achieved = sa_flops / (sa_avg_ms * 1e-3) / 1e12 if sa_n else None
+    peak = peaks["bf16_tflops_sustained"]
+    result = {
+        "metric": METRIC,
+        "value": world * B * L / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic latents/contexts, random-init bf16 weights of the named shapes",
+        "config": {"workload": args.workload, "model": "Wan2.1-T2V-1.3B shape" if "1.3b" in args.workload else cfg,
+                   "global_batch": world * B, "seq_len": L, "text_len": Lc, "blocks": cfg["num_blocks"],
+                   "timesteps": w["timesteps"], "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (2.8 GB weights + GBs of activations per step); no flush"},
+        "tflops_per_step": flops / 1e12,
+        "achieved_tflops": flops / (ms * 1e-3) / 1e12,
+        "tc_peak_frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "tc_peak_frac_of": f"{peaks['source']} bf16 {peaks['bf16_tflops']} TFLOP/s (burst)",
+        "roofline": {"kernel": "self-attention (attn_tc_kernel)", "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None,
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "flops_per_launch": sa_flops, "avg_launch_ms": sa_avg_ms, "launches_per_step": sa_n,
+                     "traffic": None},
+        "kernel_ms_per_step": {c: v[0] for c, v in kt.items()},
+        "e2e": {"value": world * B * L / (ms_e2e * 1e-3), "unit": "tokens/s", "ms_per_step": ms_e2e,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk,
+    }
+    return result
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=6)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        from video_diffusion_transformer_dit_b200 import configs
+        import torch
+        w = configs.workload(args.workload)
+        vals = []
+        for k in range(args.warmup + args.steps):
+            tok_s, step_s, desc, spent = cpu_sample(w)
+            if k >= args.warmup:
+                vals.append((tok_s, step_s))
+        tok_s = sum(v[0] for v in vals) / len(vals)
+        step_s = sum(v[1] for v in vals) / len(vals)
+        cores = torch.get_num_threads()
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload},
+            "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                w = __import__("video_diffusion_transformer_dit_b200.configs", fromlist=["x"]).workload(args.workload)
+                tok_s, step_s, desc, _ = cpu_sample(w)
+                res["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": torch.get_num_threads(),
+                                       "kind": "oracle", "sample": desc}
+            print(json.dumps(res))
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,114 @@
+/*
+ * wandit_ops.h -- kernel-level entry points of libwandit.so.
+ *
+ * These launch, one at a time, the same sm_100a kernels that wan_dit_forward()
+ * strings together, so each step of the Wan DiT forward can be checked on its
+ * own.  Citations name the page and section whose computation the kernel
+ * performs (see wandit.h for the page list).  Conventions are those of
+ * wandit.h: plain device pointers, `stream` is a cudaStream_t as void*, calls
+ * are asynchronous, nothing is retained after the call, shape errors are
+ * reported before any launch, and wan_op_sync() reports a kernel wait that ran
+ * out of time.  All matrices are dense row-major with the given leading
+ * dimension (in elements); bf16 means IEEE bfloat16, f32 means float.
+ */
+#ifndef WANDIT_OPS_H
+#define WANDIT_OPS_H
+
+#include <stdint.h>
+#include "wandit.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* GEMM epilogues: out[r, c] for acc = sum_k A[r, k] * W[c, k] (fp32 in TMEM).
+ *  WAN_EPI_BIAS          out bf16 = acc + bias[c]                       (every nn.Linear)
+ *  WAN_EPI_BIAS_GELU     out bf16 = GELU_tanh(acc + bias[c])            (ffn.net.0 + activation;
+ *                        text_embedder linear_1 + activation)
+ *  WAN_EPI_GATE_RESIDUAL out bf16 = out + (acc + bias[c]) * gate(r, c)  ("hidden_states.float()
+ *                        + attn_output * gate_msa" / "+ ff_output * c_gate_msa" in
+ *                        WanTransformerBlock), gate(r, c) = gate0[c] + gate1[(r / mod_div) * mod_ld + c]
+ *  WAN_EPI_RESIDUAL      out bf16 = out + bf16(acc + bias[c])           (cross-attention residual)
+ *  WAN_EPI_BIAS_F32      out f32  = acc + bias[c]
+ *  WAN_EPI_UNPATCHIFY    velocity f32 = bf16(acc + bias[c]) scattered by the unpatchify map
+ *                        (WanTransformer3DModel step 5); row r = b * L + token, column
+ *                        c = ((kt * ph + kh) * pw + kw) * up_C + ch.                      */
+enum {
+    WAN_EPI_BIAS = 0,
+    WAN_EPI_BIAS_GELU = 1,
+    WAN_EPI_GATE_RESIDUAL = 2,
+    WAN_EPI_RESIDUAL = 3,
+    WAN_EPI_BIAS_F32 = 4,
+    WAN_EPI_UNPATCHIFY = 5
+};
+
+typedef struct {
+    const float* bias;    /* [N] f32, or NULL for no bias                         */
+    void* out;            /* output (bf16 or f32 per epilogue); read too for the
+                             residual epilogues                                  */
+    int64_t ldo;          /* row stride of out in elements                        */
+    const float* gate0;   /* [N] f32 (gate epilogue)                              */
+    const float* gate1;   /* f32 rows of the per-sample / per-token modulation    */
+    int mod_div;          /* modulation row = r / mod_div                         */
+    int64_t mod_ld;       /* row stride of gate1 in elements                      */
+    int up_C, up_F, up_Hz, up_Wz; /* unpatchify geometry, patch (1,2,2)           */
+} wan_epilogue;
+
+/* C = epilogue(A[M,K] . W[N,K]^T).  A, W bf16 device pointers, 16-byte aligned
+ * rows (lda, ldw multiples of 8).  Requires K % 64 == 0 and N % 64 == 0; M is
+ * arbitrary (ragged last tile masked).  tcgen05 MMA with TMEM accumulators fed
+ * by TMA.                                                                   */
+WANDIT_API wan_status wan_op_gemm(const void* A, int64_t lda, const void* W, int64_t ldw,
+                       int M, int N, int K, int epilogue, const wan_epilogue* epi, void* stream);
+
+/* Flash attention O = softmax(Q K^T / sqrt(128)) V per (batch, head), no mask
+ * ("WanTransformerBlock" attn1 / attn2; bidirectional full attention,
+ * 【VLA与模仿学习】Wan2.1框架与训练源码导读 §5.2).  Row (b, l) of Q/O starts at
+ * q + (b * Lq + l) * ldq; of K/V at k + (b * Lk + l) * ldk; head h occupies
+ * columns [128 h, 128 h + 128).  bf16 in/out, fp32 online softmax.          */
+WANDIT_API wan_status wan_op_attention(const void* q, int64_t ldq, const void* k, int64_t ldk,
+                            const void* v, int64_t ldv, void* o, int64_t ldo,
+                            int B, int heads, int Lq, int Lk, void* stream);
+
+/* LayerNorm of bf16 rows x[rows, D] (fp32 statistics, biased variance, eps),
+ * then either an affine (gamma, beta; mode 1: norm2) or the adaLN modulation
+ * (mode 0: y = LN(x) * (1 + scale0[c] + scale1[m c]) + shift0[c] + shift1[m c],
+ * m = r / mod_div, row stride mod_ld; norm1/norm3/norm_out).  Output bf16.  */
+WANDIT_API wan_status wan_op_layernorm(const void* x, void* y, int rows, int D, float eps, int mode,
+                            const float* gamma, const float* beta,
+                            const float* shift0, const float* shift1,
+                            const float* scale0, const float* scale1,
+                            int mod_div, int64_t mod_ld, void* stream);
+
+/* In-place RMSNorm across all heads of bf16 row segments buf[r, 0:D] (row
+ * stride ld), times gain[D] ("qk_norm = rms_norm_across_heads"), then, when
+ * rope != 0, the 3-axis rotary embedding of token l = r % (Fp*Hp*Wp) at grid
+ * position (f, i, j) (RoPE per T/H/W axis, pairs (2k, 2k+1) of each 128-wide
+ * head, head-dim split rope_t/h/w, base theta).                             */
+WANDIT_API wan_status wan_op_rmsnorm_rope(void* buf, int64_t ld, int rows, int D, float eps, const float* gain,
+                               int rope, int Fp, int Hp, int Wp, int rope_t, int rope_h, int rope_w,
+                               float theta, void* stream);
+
+/* Patchify gather: latent [B, C, F, Hz, Wz] (f32 or bf16) -> X bf16
+ * [B * L, C * 4] with token order (f, i, j) and feature order (c, kh, kw) --
+ * the input view of patch_embedding = Conv3d(k = s = (1,2,2)).               */
+WANDIT_API wan_status wan_op_patchify(const void* latent, int latent_dtype, int B, int C, int F, int Hz, int Wz,
+                           void* X, void* stream);
+
+/* Unpatchify scatter: rows f32 [B * L, 4 * C] (feature order (kh, kw, c)) ->
+ * velocity f32 [B, C, F, Hz, Wz]; the same index map the proj_out epilogue
+ * uses.                                                                     */
+WANDIT_API wan_status wan_op_unpatchify(const float* rows, int B, int C, int F, int Hz, int Wz,
+                             float* velocity, void* stream);
+
+/* Synchronise `stream`; WAN_ETIMEOUT if an op kernel's bounded wait ran out
+ * (flag cleared), WAN_ECUDA on a CUDA error.                                */
+WANDIT_API wan_status wan_op_sync(void* stream);
+
+/* Time limit in ns of every on-chip wait of the op kernels (default 2e9). */
+WANDIT_API void wan_op_set_wait_limit_ns(int64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WANDIT_OPS_H */

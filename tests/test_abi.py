@@ -1,0 +1,61 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds, loads,
+exports every entry point include/*.h declares, and rejects configurations
+the kernels do not cover before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from video_diffusion_transformer_dit_b200 import binding, build
+    build.build()
+    return binding.lib()
+
+
+def declared_symbols():
+    names = set()
+    for h in ("wandit.h", "wandit_ops.h"):
+        text = open(os.path.join(ROOT, "include", h)).read()
+        names |= set(re.findall(r"WANDIT_API\s+[\w\s\*]+?\b(wan_\w+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from video_diffusion_transformer_dit_b200 import binding
+    names = declared_symbols()
+    assert len(names) >= 20
+    assert names == set(binding.SYMBOLS)
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_status_strings(lib):
+    for code in range(11):
+        s = lib.wan_status_string(code)
+        assert s and s.decode() != "unknown status"
+
+
+def test_create_rejects_unsupported_configs_without_a_device(lib):
+    from video_diffusion_transformer_dit_b200 import binding, configs
+    base = configs.model_config("wan2.1-1.3b")
+    bad = [dict(base, head_dim=64, heads=24), dict(base, dim=1000), dict(base, patch=(2, 2, 2)),
+           dict(base, rope_split=(44, 42, 40)), dict(base, ffn_dim=100)]
+    for cfg in bad:
+        c = binding.make_config(cfg, 1, 192, 32)
+        h = ctypes.c_void_p()
+        assert lib.wan_dit_create(ctypes.byref(c), 0, ctypes.byref(h)) == 10   # WAN_EUNSUPPORTED
+        assert not h
+    h = ctypes.c_void_p()
+    assert lib.wan_dit_create(None, 0, ctypes.byref(h)) == 1                   # WAN_EINVAL
+
+
+def test_null_handle_calls_are_refused(lib):
+    assert lib.wan_dit_forward(None, None, 0, 1, 1, 2, 2, None, 0, None, 1, None, 1, None) == 1
+    assert lib.wan_dit_sync(None, None) == 1
+    assert lib.wan_dit_last_launch_count(None) == 0
+    assert lib.wan_dit_last_error(None) == b"null handle"

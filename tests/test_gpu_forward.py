@@ -1,0 +1,160 @@
+"""Whole-forward parity of wan_dit_forward against the float64 oracle.
+
+* one block + head at 192 tokens: every element, with the per-block error
+  report (the residual stream after the patch embedding and after the block);
+* the per-token-timestep variant (Wan2.2-5B widths, 48 channels);
+* the 480p CFG-batch shapes (B = 2, L = 32760, launch configuration of the
+  benchmark) with one block: sampled tokens against the oracle's row mode;
+* the same shapes with all 30 blocks: properties that hold at any size
+  (identical samples give identical outputs, run-to-run determinism, graph
+  replay equals eager launches, finite values);
+* argument validation and weight bookkeeping of the C ABI.
+Tolerance on the velocity: relative L2 <= 2e-2 (bf16 storage, fp32
+accumulation), the bound the method's precision policy allows.
+"""
+import pytest
+import torch
+
+from oracle import wan_oracle as O
+from tests.gpu_common import DT, make_dit, need_gpu, rel_l2, to64, workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+
+
+def report(tag, errs):
+    print(f"\n[{tag}] per-block rel-L2: " + " ".join(f"{e:.2e}" for e in errs))
+
+
+def run_gpu(dit, lat, t, ctx):
+    v = dit.forward(lat.cuda(), t.cuda(), ctx.cuda(), sync=True)
+    return v.cpu()
+
+
+def test_forward_one_block_192_tokens():
+    cfg, W, lat, t, ctx = workload_inputs("wan1.3b-1blk-3x16x16")
+    B, L, Lc = 1, O.token_count(*lat.shape[2:]), ctx.shape[1]
+    dit = make_dit(cfg, B, L, Lc, W)
+    dump = torch.zeros(cfg["num_blocks"] + 1, B * L, cfg["dim"], dtype=torch.bfloat16, device="cuda")
+    dit.set_block_dump(dump)
+    v_eager = run_gpu(dit, lat, t, ctx)
+    dit.set_block_dump(None)
+    ref, blocks = O.forward(lat.to(DT), t.to(DT), ctx.to(DT), to64(W), cfg, return_blocks=True)
+    errs = [rel_l2(dump[i].cpu(), blocks[i].reshape(B * L, -1)) for i in range(len(blocks))]
+    report("1 block, 192 tokens", errs)
+    assert max(errs) < TOL
+    err = rel_l2(v_eager, ref)
+    print(f"velocity rel-L2 {err:.3e}")
+    assert err < TOL
+    # graph replay == eager launches, bit for bit, and run to run
+    v_graph = run_gpu(dit, lat, t, ctx)
+    v_graph2 = run_gpu(dit, lat, t, ctx)
+    assert torch.equal(v_graph, v_eager)
+    assert torch.equal(v_graph, v_graph2)
+    assert dit.last_launch_count() > 0
+
+
+def test_forward_host_io_matches_device_io():
+    cfg, W, lat, t, ctx = workload_inputs("wan1.3b-1blk-3x16x16", seed=1)
+    B, L, Lc = 1, O.token_count(*lat.shape[2:]), ctx.shape[1]
+    dit = make_dit(cfg, B, L, Lc, W)
+    v_dev = run_gpu(dit, lat, t, ctx)
+    v_host = dit.forward(lat.pin_memory(), t.pin_memory(), ctx.pin_memory())
+    dit.sync()
+    assert not v_host.is_cuda
+    assert torch.equal(v_host, v_dev)
+
+
+def test_forward_per_token_timestep_5b_widths():
+    from video_diffusion_transformer_dit_b200 import configs, synth
+    cfg = configs.model_config("wan2.2-5b", num_blocks=1)
+    shape = (1, 48, 3, 16, 16)
+    L = O.token_count(*shape[2:])
+    W = synth.make_weights(cfg, seed=3)
+    lat = synth.make_latent(shape, seed=3)
+    ctx = synth.make_context(1, 40, cfg["text_dim"], seed=3)
+    t = synth.make_timestep_per_token(1, L, 64, seed=3)
+    dit = make_dit(cfg, 1, L, 40, W)
+    v = run_gpu(dit, lat, t, ctx)
+    ref = O.forward(lat.to(DT), t.to(DT), ctx.to(DT), to64(W), cfg)
+    err = rel_l2(v, ref)
+    print(f"\nper-token 5B widths velocity rel-L2 {err:.3e}")
+    assert err < TOL
+
+
+def test_forward_480p_cfg_batch_one_block_sampled_rows():
+    """B = 2, L = 32760 (81 frames 480x832), one block: sampled tokens of both
+    samples against the oracle's row mode (keys/values over every token)."""
+    cfg, W, lat, t, ctx = workload_inputs("wan1.3b-81f-480x832-cfg2", num_blocks=1)
+    B, Cc, F, Hz, Wz = lat.shape
+    L, Lc = O.token_count(F, Hz, Wz), ctx.shape[1]
+    dit = make_dit(cfg, B, L, Lc, W)
+    v = run_gpu(dit, lat, t, ctx)
+    g = torch.Generator().manual_seed(0)
+    rows = torch.cat([torch.tensor([0, 1, L // 2, L - 1]), torch.randint(0, L, (60,), generator=g)]).unique()
+    o = O.forward(lat.to(DT), t.to(DT), ctx.to(DT), to64(W), cfg, rows=rows)
+    idx = O.unpatch_index_map(Cc, F, Hz, Wz)[rows]
+    got = v.reshape(B, -1)[:, idx]
+    err = rel_l2(got, o)
+    print(f"\n480p B=2 one block, {rows.numel()} sampled tokens rel-L2 {err:.3e}")
+    assert err < TOL
+
+
+def test_forward_480p_cfg_batch_30_blocks_properties():
+    cfg, W, lat, t, ctx = workload_inputs("wan1.3b-81f-480x832-cfg2")
+    B, Cc, F, Hz, Wz = lat.shape
+    L, Lc = O.token_count(F, Hz, Wz), ctx.shape[1]
+    dit = make_dit(cfg, B, L, Lc, W)
+    ctx_same = ctx[:1].expand(B, -1, -1).contiguous()
+    v1 = run_gpu(dit, lat, t, ctx_same)
+    assert torch.isfinite(v1).all()
+    assert torch.equal(v1[0], v1[1])            # identical samples, identical outputs
+    v2 = run_gpu(dit, lat, t, ctx_same)
+    assert torch.equal(v1, v2)                  # deterministic
+    v3 = run_gpu(dit, lat, t, ctx)              # two contexts: the samples differ
+    assert torch.isfinite(v3).all()
+    assert not torch.equal(v3[0], v3[1])
+    assert 0.1 < v3.std().item() < 10.0
+
+
+# ------------------------------------------------------------------ C ABI bookkeeping
+def test_abi_validation_and_missing_weights():
+    from video_diffusion_transformer_dit_b200.binding import WanError
+    cfg, W, lat, t, ctx = workload_inputs("wan1.3b-1blk-3x16x16", seed=2)
+    L, Lc = O.token_count(*lat.shape[2:]), ctx.shape[1]
+    dit = make_dit(cfg, 1, L, Lc)
+    with pytest.raises(WanError) as e:
+        dit.forward(lat.cuda(), t.cuda(), ctx.cuda())
+    assert e.value.name == "WAN_ENOWEIGHTS"
+    part = {k: v.cuda() for k, v in W.items() if k != "proj_out.bias"}
+    dit.load_weights(part)
+    n, names = dit.missing_weights()
+    assert n == 1 and names == "proj_out.bias"
+    with pytest.raises(WanError) as e:
+        dit.forward(lat.cuda(), t.cuda(), ctx.cuda())
+    assert e.value.name == "WAN_EMISSING_WEIGHT"
+    with pytest.raises(WanError) as e:
+        dit.load_weights({"blocks.7.attn1.to_q.weight": W["blocks.0.attn1.to_q.weight"].cuda()})
+    assert e.value.name == "WAN_EUNEXPECTED_WEIGHT"
+    with pytest.raises(WanError) as e:
+        dit.load_weights({"proj_out.bias": torch.zeros(63, device="cuda")})
+    assert e.value.name == "WAN_ESHAPE"
+    dit.load_weights({"proj_out.bias": W["proj_out.bias"].cuda()})
+    assert dit.missing_weights()[0] == 0
+    # shapes beyond the workspace limits or odd grids are refused before any launch
+    big = torch.zeros(1, 16, 4, 16, 16, device="cuda")
+    with pytest.raises(WanError) as e:
+        dit.forward(big, t.cuda(), ctx.cuda())
+    assert e.value.name == "WAN_ESHAPE"
+    odd = torch.zeros(1, 16, 3, 15, 16, device="cuda")
+    with pytest.raises(WanError) as e:
+        dit.forward(odd, t.cuda(), ctx.cuda())
+    assert e.value.name == "WAN_ESHAPE"
+    v = dit.forward(lat.cuda(), t.cuda(), ctx.cuda(), sync=True)
+    assert torch.isfinite(v).all()

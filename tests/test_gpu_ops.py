@@ -1,0 +1,245 @@
+"""Kernel-level parity: each CUDA kernel through the C ABI against the oracle.
+
+Index maps (patchify / unpatchify) must match bit for bit; floating-point
+kernels are compared by relative L2 error against float64 (bf16 storage with
+fp32 accumulation: 1e-2 bounds a few bf16 roundings, 2^-9 each).
+"""
+import math
+
+import pytest
+import torch
+
+from oracle import wan_oracle as O
+from tests.gpu_common import DT, bf16_round, need_gpu, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+    from video_diffusion_transformer_dit_b200 import binding
+    binding.lib()
+
+
+def B():
+    from video_diffusion_transformer_dit_b200 import binding
+    return binding
+
+
+# ------------------------------------------------------------------ index maps
+@pytest.mark.parametrize("shape", [(1, 16, 3, 16, 16), (2, 16, 9, 44, 80), (1, 48, 2, 10, 6)])
+def test_patchify_bit_exact(shape):
+    lat = bf16_round(torch.randn(*shape))
+    X = torch.empty(shape[0] * O.token_count(*shape[2:]), shape[1] * 4, dtype=torch.bfloat16, device="cuda")
+    B().op_patchify(lat.cuda(), X)
+    B().op_sync()
+    ref = O.patchify(lat.to(DT)).reshape(X.shape)
+    assert torch.equal(X.cpu().to(DT), ref)
+
+
+def test_patchify_bf16_latent_bit_exact():
+    lat = torch.randn(2, 16, 3, 8, 12).to(torch.bfloat16)
+    X = torch.empty(2 * 3 * 4 * 6, 64, dtype=torch.bfloat16, device="cuda")
+    B().op_patchify(lat.cuda(), X)
+    B().op_sync()
+    assert torch.equal(X.cpu().to(DT), O.patchify(lat.to(DT)).reshape(X.shape))
+
+
+@pytest.mark.parametrize("shape", [(1, 16, 3, 16, 16), (2, 16, 21, 60, 104), (1, 48, 3, 44, 80)])
+def test_unpatchify_bit_exact(shape):
+    Bn, Cc, F, Hz, Wz = shape
+    L = O.token_count(F, Hz, Wz)
+    rows = torch.randn(Bn * L, 4 * Cc)
+    vel = torch.full(shape, float("nan"), device="cuda")
+    B().op_unpatchify(rows.cuda(), vel)
+    B().op_sync()
+    ref = O.unpatchify(rows.reshape(Bn, L, 4 * Cc).to(DT), Cc, F, Hz, Wz)
+    assert torch.equal(vel.cpu().to(DT), ref)
+
+
+# ------------------------------------------------------------------ GEMM
+def _gemm_inputs(M, N, K, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g)
+    return A, W, bias
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 256, 192), (1000, 1536, 1536), (129, 128, 64), (77, 64, 256),
+                                   (4100, 4608, 1536), (452, 9216, 1536)])
+def test_gemm_bias(M, N, K):
+    A, W, bias = _gemm_inputs(M, N, K)
+    out = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    B().op_gemm(A.cuda(), W.cuda(), "bias", out, bias=bias.cuda())
+    B().op_sync()
+    ref = O.linear(A.to(DT), W.to(DT), bias.to(DT))
+    assert rel_l2(out, ref) < TOL
+
+
+def test_gemm_bias_gelu_and_f32():
+    M, N, K = 333, 512, 320
+    A, W, bias = _gemm_inputs(M, N, K, seed=1)
+    out = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    B().op_gemm(A.cuda(), W.cuda(), "bias_gelu", out, bias=bias.cuda())
+    out32 = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+    B().op_gemm(A.cuda(), W.cuda(), "bias_f32", out32, bias=bias.cuda())
+    B().op_sync()
+    lin = O.linear(A.to(DT), W.to(DT), bias.to(DT))
+    assert rel_l2(out, O.gelu_tanh(lin)) < TOL
+    assert rel_l2(out32, lin) < 1e-4
+
+
+@pytest.mark.parametrize("per_token", [False, True])
+def test_gemm_gate_residual(per_token):
+    M, N, K, L = 400, 256, 256, 200          # two samples of 200 tokens
+    A, W, bias = _gemm_inputs(M, N, K, seed=2)
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(M, N, generator=g).to(torch.bfloat16)
+    sst = torch.randn(6, N, generator=g) * 0.1
+    rows_mod = M if per_token else 2
+    tproj = torch.randn(rows_mod, 6, N, generator=g) * 0.1
+    xd = x.cuda()
+    B().op_gemm(A.cuda(), W.cuda(), "gate_residual", xd, bias=bias.cuda(), gate0=sst[2].contiguous().cuda(),
+                gate1=tproj[:, 2].contiguous().cuda(), mod_div=1 if per_token else L, mod_ld=N)
+    B().op_sync()
+    gate = sst[2].to(DT) + (tproj[:, 2].to(DT) if per_token else tproj[:, 2].to(DT).repeat_interleave(L, 0))
+    ref = x.to(DT) + O.linear(A.to(DT), W.to(DT), bias.to(DT)) * gate
+    assert rel_l2(xd, ref) < TOL
+
+
+def test_gemm_residual():
+    M, N, K = 260, 384, 128
+    A, W, bias = _gemm_inputs(M, N, K, seed=4)
+    x = torch.randn(M, N).to(torch.bfloat16)
+    xd = x.cuda()
+    B().op_gemm(A.cuda(), W.cuda(), "residual", xd, bias=bias.cuda())
+    B().op_sync()
+    ref = x.to(DT) + O.linear(A.to(DT), W.to(DT), bias.to(DT))
+    assert rel_l2(xd, ref) < TOL
+
+
+@pytest.mark.parametrize("shape", [(1, 16, 3, 16, 16), (2, 16, 5, 12, 20), (1, 48, 2, 8, 8)])
+def test_gemm_unpatchify_epilogue(shape):
+    Bn, Cc, F, Hz, Wz = shape
+    L = O.token_count(F, Hz, Wz)
+    M, N, K = Bn * L, 4 * Cc, 256
+    A, W, bias = _gemm_inputs(M, N, K, seed=5)
+    vel = torch.full(shape, float("nan"), device="cuda")
+    B().op_gemm(A.cuda(), W.cuda(), "unpatchify", vel, bias=bias.cuda(), unpatch=(Cc, F, Hz, Wz))
+    B().op_sync()
+    o = O.linear(A.to(DT), W.to(DT), bias.to(DT)).reshape(Bn, L, N)
+    ref = O.unpatchify(o, Cc, F, Hz, Wz)
+    assert not torch.isnan(vel).any()
+    assert rel_l2(vel, ref) < TOL
+
+
+def test_gemm_rejects_bad_shapes():
+    from video_diffusion_transformer_dit_b200.binding import WanError
+    A = torch.zeros(64, 100, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(64, 100, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(WanError):
+        B().op_gemm(A, W, "bias", out)
+
+
+# ------------------------------------------------------------------ attention
+@pytest.mark.parametrize("Bn,heads,Lq,Lk", [(1, 1, 128, 128), (2, 2, 300, 300), (2, 3, 200, 226),
+                                            (1, 2, 1000, 32), (1, 1, 5, 700)])
+def test_attention(Bn, heads, Lq, Lk):
+    D = heads * 128
+    g = torch.Generator().manual_seed(Lq * 7 + Lk)
+    q = torch.randn(Bn * Lq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(Bn * Lk, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(Bn * Lk, D, generator=g).to(torch.bfloat16)
+    o = torch.zeros(Bn * Lq, D, dtype=torch.bfloat16, device="cuda")
+    B().op_attention(q.cuda(), k.cuda(), v.cuda(), o, Bn, heads, Lq, Lk)
+    B().op_sync()
+    ref = O.attention(q.to(DT).reshape(Bn, Lq, heads, 128), k.to(DT).reshape(Bn, Lk, heads, 128),
+                      v.to(DT).reshape(Bn, Lk, heads, 128)).reshape(Bn * Lq, D)
+    assert rel_l2(o, ref) < TOL
+
+
+def test_attention_strided_qkv_buffer():
+    """q, k, v as column slices of one [rows, 3D] buffer, as the forward uses them."""
+    Bn, heads, L = 2, 2, 260
+    D = heads * 128
+    qkv = torch.randn(Bn * L, 3 * D).to(torch.bfloat16)
+    d = qkv.cuda()
+    o = torch.zeros(Bn * L, D, dtype=torch.bfloat16, device="cuda")
+    base = d.data_ptr()
+    B().op_attention_ptr(base, 3 * D, base + 2 * D, 3 * D, base + 4 * D, 3 * D, o.data_ptr(), D, Bn, heads, L, L)
+    B().op_sync()
+    t = qkv.to(DT).reshape(Bn, L, 3, heads, 128)
+    ref = O.attention(t[:, :, 0], t[:, :, 1], t[:, :, 2]).reshape(Bn * L, D)
+    assert rel_l2(o, ref) < TOL
+
+
+def test_attention_large_logits_rescale():
+    """Keys whose logits grow along the sequence force the running-max rescale."""
+    Bn, heads, Lq, Lk = 1, 1, 128, 1024
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn(Lq, 128, generator=g)
+    k = torch.randn(Lk, 128, generator=g) * torch.linspace(0.1, 4.0, Lk)[:, None]
+    v = torch.randn(Lk, 128, generator=g)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    o = torch.zeros(Lq, 128, dtype=torch.bfloat16, device="cuda")
+    B().op_attention(q.cuda(), k.cuda(), v.cuda(), o, Bn, heads, Lq, Lk)
+    B().op_sync()
+    ref = O.attention(q.to(DT)[None, :, None], k.to(DT)[None, :, None], v.to(DT)[None, :, None])[0, :, 0]
+    assert rel_l2(o, ref) < TOL
+
+
+# ------------------------------------------------------------------ norms
+@pytest.mark.parametrize("D", [1536, 3072, 5120])
+def test_layernorm_modulated(D):
+    rows, L = 600, 300
+    g = torch.Generator().manual_seed(D)
+    x = (torch.randn(rows, D, generator=g) * 2 + 0.5).to(torch.bfloat16)
+    sst = torch.randn(6, D, generator=g) * 0.2
+    tproj = torch.randn(2, 6, D, generator=g) * 0.2
+    y = torch.zeros_like(x, device="cuda")
+    tp = tproj.reshape(2, 6 * D).contiguous().cuda()
+    s = sst.cuda()
+    B().op_layernorm(x.cuda(), y, 1e-6, 0, shift0=s[0], shift1=tp[:, 0:D], scale0=s[1], scale1=tp[:, D:2 * D],
+                     mod_div=L, mod_ld=6 * D)
+    B().op_sync()
+    shift = sst[0].to(DT) + tproj[:, 0].to(DT).repeat_interleave(L, 0)
+    scale = sst[1].to(DT) + tproj[:, 1].to(DT).repeat_interleave(L, 0)
+    ref = O.layer_norm(x.to(DT), 1e-6) * (1 + scale) + shift
+    assert rel_l2(y, ref) < TOL
+
+
+def test_layernorm_affine():
+    rows, D = 333, 1536
+    x = torch.randn(rows, D).to(torch.bfloat16)
+    gam = 1 + torch.randn(D) * 0.1
+    bet = torch.randn(D) * 0.1
+    y = torch.zeros_like(x, device="cuda")
+    B().op_layernorm(x.cuda(), y, 1e-6, 1, gamma=gam.cuda(), beta=bet.cuda())
+    B().op_sync()
+    assert rel_l2(y, O.layer_norm(x.to(DT), 1e-6, gam.to(DT), bet.to(DT))) < TOL
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_rmsnorm_rope(rope):
+    Fp, Hp, Wp = 3, 5, 7
+    L = Fp * Hp * Wp
+    Bn, D = 2, 1536
+    ld = 3 * D
+    buf = torch.randn(Bn * L, ld).to(torch.bfloat16)
+    gain = 1 + torch.randn(D) * 0.1
+    d = buf.cuda()
+    B().op_rmsnorm_rope(d.data_ptr() + 2 * D, ld, Bn * L, D, 1e-6, gain.cuda(), rope=rope, grid=(Fp, Hp, Wp))
+    B().op_sync()
+    seg = buf[:, D:2 * D].to(DT)
+    ref = O.rms_norm(seg, 1e-6, gain.to(DT))
+    if rope:
+        ang = O.rope_angles((Fp, Hp, Wp), (44, 42, 42), 10000.0)
+        ref = O.rope_apply(ref.reshape(Bn, L, 12, 128), ang).reshape(Bn * L, D)
+    got = d.cpu()
+    assert rel_l2(got[:, D:2 * D], ref) < TOL
+    assert torch.equal(got[:, :D], buf[:, :D]) and torch.equal(got[:, 2 * D:], buf[:, 2 * D:])

@@ -1,0 +1,287 @@
+"""Thin ctypes binding of libwandit.so (include/wandit.h, include/wandit_ops.h).
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels.  PyTorch tensors are passed by their ``data_ptr()``; streams by
+``torch.cuda.current_stream().cuda_stream``.  Loading raises if the library has
+not been built (``python -m video_diffusion_transformer_dit_b200.build``):
+there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Dict, Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwandit.so")
+
+WAN_STATUS = {0: "WAN_OK", 1: "WAN_EINVAL", 2: "WAN_ESHAPE", 3: "WAN_ENOMEM", 4: "WAN_ENOWEIGHTS",
+              5: "WAN_EMISSING_WEIGHT", 6: "WAN_EUNEXPECTED_WEIGHT", 7: "WAN_ECUDA", 8: "WAN_ETIMEOUT",
+              9: "WAN_EINTERNAL", 10: "WAN_EUNSUPPORTED"}
+WAN_DTYPE_F32, WAN_DTYPE_BF16 = 0, 1
+WAN_OPT_GRAPH, WAN_OPT_WAIT_LIMIT_NS, WAN_OPT_KERNEL_TIMING = 1, 2, 3
+KERNEL_CLASSES = {"patchify": 0, "gemm": 1, "self_attention": 2, "cross_attention": 3, "layernorm": 4,
+                  "rmsnorm_rope": 5, "embedding": 6}
+EPI = {"bias": 0, "bias_gelu": 1, "gate_residual": 2, "residual": 3, "bias_f32": 4, "unpatchify": 5}
+
+# every symbol include/*.h declares
+SYMBOLS = ["wan_dit_create", "wan_dit_load_weights", "wan_dit_missing_weights", "wan_dit_forward", "wan_dit_sync",
+           "wan_dit_set_block_dump", "wan_dit_set_option", "wan_dit_kernel_time", "wan_dit_last_launch_count",
+           "wan_dit_flops",
+           "wan_dit_last_error", "wan_status_string", "wan_dit_destroy",
+           "wan_op_gemm", "wan_op_attention", "wan_op_layernorm", "wan_op_rmsnorm_rope", "wan_op_patchify",
+           "wan_op_unpatchify", "wan_op_sync", "wan_op_set_wait_limit_ns"]
+
+
+class WanError(RuntimeError):
+    def __init__(self, status: int, msg: str = ""):
+        self.status = status
+        self.name = WAN_STATUS.get(status, str(status))
+        super().__init__(f"{self.name}: {msg}")
+
+
+class wan_dit_config(C.Structure):
+    _fields_ = [(n, C.c_int) for n in ("dim", "heads", "head_dim", "ffn_dim", "num_blocks", "in_ch", "out_ch",
+                                        "patch_t", "patch_h", "patch_w", "text_dim", "freq_dim",
+                                        "rope_t", "rope_h", "rope_w")] + \
+              [("eps", C.c_float), ("rope_theta", C.c_float)] + \
+              [(n, C.c_int) for n in ("max_batch", "max_tokens", "max_text")]
+
+
+class wan_epilogue(C.Structure):
+    _fields_ = [("bias", C.c_void_p), ("out", C.c_void_p), ("ldo", C.c_int64), ("gate0", C.c_void_p),
+                ("gate1", C.c_void_p), ("mod_div", C.c_int), ("mod_ld", C.c_int64),
+                ("up_C", C.c_int), ("up_F", C.c_int), ("up_Hz", C.c_int), ("up_Wz", C.c_int)]
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libwandit.so (once) and declare its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise FileNotFoundError(f"{LIB_PATH} is missing: build it with "
+                                "`python -m video_diffusion_transformer_dit_b200.build`")
+    L = C.CDLL(LIB_PATH)
+    P, I, I64, D, F = C.c_void_p, C.c_int, C.c_int64, C.c_double, C.c_float
+    sig = {
+        "wan_dit_create": (I, [C.POINTER(wan_dit_config), I, C.POINTER(P)]),
+        "wan_dit_load_weights": (I, [P, I, C.POINTER(C.c_char_p), C.POINTER(P), C.POINTER(I),
+                                     C.POINTER(C.POINTER(I64)), C.POINTER(I), I, P]),
+        "wan_dit_missing_weights": (I, [P, C.c_char_p, I]),
+        "wan_dit_forward": (I, [P, P, I, I, I, I, I, P, I, P, I, P, I, P]),
+        "wan_dit_sync": (I, [P, P]),
+        "wan_dit_set_block_dump": (I, [P, P]),
+        "wan_dit_set_option": (I, [P, I, I64]),
+        "wan_dit_kernel_time": (I, [P, I, C.POINTER(D), C.POINTER(I)]),
+        "wan_dit_last_launch_count": (I, [P]),
+        "wan_dit_flops": (D, [P, I, I, I, I, I, I]),
+        "wan_dit_last_error": (C.c_char_p, [P]),
+        "wan_status_string": (C.c_char_p, [I]),
+        "wan_dit_destroy": (None, [P]),
+        "wan_op_gemm": (I, [P, I64, P, I64, I, I, I, I, C.POINTER(wan_epilogue), P]),
+        "wan_op_attention": (I, [P, I64, P, I64, P, I64, P, I64, I, I, I, I, P]),
+        "wan_op_layernorm": (I, [P, P, I, I, F, I, P, P, P, P, P, P, I, I64, P]),
+        "wan_op_rmsnorm_rope": (I, [P, I64, I, I, F, P, I, I, I, I, I, I, I, F, P]),
+        "wan_op_patchify": (I, [P, I, I, I, I, I, I, P, P]),
+        "wan_op_unpatchify": (I, [P, I, I, I, I, I, P, P]),
+        "wan_op_sync": (I, [P]),
+        "wan_op_set_wait_limit_ns": (None, [I64]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> Optional[int]:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(status: int, msg: str = ""):
+    if status != 0:
+        raise WanError(status, msg)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return WAN_DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return WAN_DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def make_config(cfg: dict, max_batch: int, max_tokens: int, max_text: int) -> wan_dit_config:
+    c = wan_dit_config()
+    for k in ("dim", "heads", "head_dim", "ffn_dim", "num_blocks", "in_ch", "out_ch", "text_dim", "freq_dim"):
+        setattr(c, k, int(cfg[k]))
+    c.patch_t, c.patch_h, c.patch_w = (int(v) for v in cfg["patch"])
+    c.rope_t, c.rope_h, c.rope_w = (int(v) for v in cfg["rope_split"])
+    c.eps = float(cfg["eps"])
+    c.rope_theta = float(cfg["rope_theta"])
+    c.max_batch, c.max_tokens, c.max_text = int(max_batch), int(max_tokens), int(max_text)
+    return c
+
+
+class WanDiT:
+    """Handle of ``wan_dit``: create / load_weights / forward / sync / destroy."""
+
+    def __init__(self, cfg: dict, max_batch: int, max_tokens: int, max_text: int, device: int = 0):
+        self.cfg = dict(cfg)
+        self._h = C.c_void_p()
+        c = make_config(cfg, max_batch, max_tokens, max_text)
+        _check(lib().wan_dit_create(C.byref(c), int(device), C.byref(self._h)), "wan_dit_create")
+
+    # -- lifetime
+    def close(self):
+        if self._h:
+            lib().wan_dit_destroy(self._h)
+            self._h = C.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def last_error(self) -> str:
+        return lib().wan_dit_last_error(self._h).decode()
+
+    def _check(self, status):
+        if status != 0:
+            raise WanError(status, self.last_error())
+
+    # -- weights
+    def load_weights(self, weights: Dict[str, "object"], stream=None):
+        """Load a dict name -> torch tensor (f32 or bf16, CPU or CUDA, contiguous)."""
+        items = list(weights.items())
+        if not items:
+            return
+        on_dev = items[0][1].is_cuda
+        keep = [t.contiguous() for _, t in items]
+        if any(t.is_cuda != on_dev for t in keep):
+            raise ValueError("all tensors of one load call must be on the same side (host or device)")
+        n = len(items)
+        names = (C.c_char_p * n)(*[k.encode() for k, _ in items])
+        ptrs = (C.c_void_p * n)(*[t.data_ptr() for t in keep])
+        dts = (C.c_int * n)(*[_dtype_code(t) for t in keep])
+        shape_arrs = [(C.c_int64 * max(1, t.dim()))(*t.shape) for t in keep]
+        shapes = (C.POINTER(C.c_int64) * n)(*[C.cast(a, C.POINTER(C.c_int64)) for a in shape_arrs])
+        nd = (C.c_int * n)(*[t.dim() for t in keep])
+        st = _stream(stream) if on_dev else None
+        self._check(lib().wan_dit_load_weights(self._h, n, names, ptrs, dts, shapes, nd, int(on_dev), st))
+
+    def missing_weights(self):
+        buf = C.create_string_buffer(1 << 16)
+        n = lib().wan_dit_missing_weights(self._h, buf, len(buf))
+        return n, buf.value.decode()
+
+    # -- forward
+    def forward(self, latent, timestep, context, velocity=None, stream=None, sync=False):
+        """latent [B,C,F,Hz,Wz] f32/bf16, timestep f32 [B] or [B,L], context bf16
+        [B,Lc,text_dim].  All CUDA tensors (device I/O) or all CPU tensors (host
+        I/O, copies inside the call).  Returns the velocity tensor."""
+        import torch
+        B, Cin, F, Hz, Wz = latent.shape
+        Lc = context.shape[1]
+        per_token = int(timestep.dim() == 2)
+        on_dev = latent.is_cuda
+        if velocity is None:
+            velocity = torch.empty(B, self.cfg["out_ch"], F, Hz, Wz, dtype=torch.float32, device=latent.device,
+                                   pin_memory=not on_dev)
+        st = _stream(stream)
+        self._check(lib().wan_dit_forward(self._h, _ptr(latent), _dtype_code(latent), B, F, Hz, Wz, _ptr(timestep),
+                                          per_token, _ptr(context), Lc, _ptr(velocity), int(on_dev), st))
+        if sync:
+            self.sync(stream)
+        return velocity
+
+    def sync(self, stream=None):
+        self._check(lib().wan_dit_sync(self._h, _stream(stream)))
+
+    def set_block_dump(self, dst):
+        self._check(lib().wan_dit_set_block_dump(self._h, _ptr(dst)))
+
+    def set_option(self, option: int, value: int):
+        self._check(lib().wan_dit_set_option(self._h, option, int(value)))
+
+    def kernel_time(self, kernel_class: str):
+        """(total ms, launches) of one kernel class in the last timed forward."""
+        ms, n = C.c_double(), C.c_int()
+        self._check(lib().wan_dit_kernel_time(self._h, KERNEL_CLASSES[kernel_class], C.byref(ms), C.byref(n)))
+        return ms.value, n.value
+
+    def last_launch_count(self) -> int:
+        return lib().wan_dit_last_launch_count(self._h)
+
+    def flops(self, B, F, Hz, Wz, Lc, per_token=0) -> float:
+        return lib().wan_dit_flops(self._h, B, F, Hz, Wz, Lc, per_token)
+
+
+# ---------------------------------------------------------------- op-level wrappers
+def op_gemm(A, W, epilogue: str, out, bias=None, gate0=None, gate1=None, mod_div=1, mod_ld=0,
+            unpatch=(0, 0, 0, 0), M=None, stream=None):
+    M = A.shape[0] if M is None else M
+    N, K = W.shape
+    e = wan_epilogue(bias=_ptr(bias), out=_ptr(out), ldo=(out.stride(0) if out.dim() == 2 else 0),
+                     gate0=_ptr(gate0), gate1=_ptr(gate1), mod_div=mod_div, mod_ld=mod_ld,
+                     up_C=unpatch[0], up_F=unpatch[1], up_Hz=unpatch[2], up_Wz=unpatch[3])
+    _check(lib().wan_op_gemm(_ptr(A), A.stride(0), _ptr(W), W.stride(0), M, N, K, EPI[epilogue], C.byref(e),
+                             _stream(stream)), "wan_op_gemm")
+
+
+def op_attention(q, k, v, o, B, heads, Lq, Lk, ldq=None, ldk=None, ldv=None, ldo=None, stream=None):
+    _check(lib().wan_op_attention(_ptr(q), ldq or q.stride(0), _ptr(k), ldk or k.stride(0), _ptr(v),
+                                  ldv or v.stride(0), _ptr(o), ldo or o.stride(0), B, heads, Lq, Lk,
+                                  _stream(stream)), "wan_op_attention")
+
+
+def op_attention_ptr(q, ldq, k, ldk, v, ldv, o, ldo, B, heads, Lq, Lk, stream=None):
+    _check(lib().wan_op_attention(q, ldq, k, ldk, v, ldv, o, ldo, B, heads, Lq, Lk, _stream(stream)),
+           "wan_op_attention")
+
+
+def op_layernorm(x, y, eps, mode, gamma=None, beta=None, shift0=None, shift1=None, scale0=None, scale1=None,
+                 mod_div=1, mod_ld=0, stream=None):
+    rows, D = x.shape
+    _check(lib().wan_op_layernorm(_ptr(x), _ptr(y), rows, D, eps, mode, _ptr(gamma), _ptr(beta), _ptr(shift0),
+                                  _ptr(shift1), _ptr(scale0), _ptr(scale1), mod_div, mod_ld, _stream(stream)),
+           "wan_op_layernorm")
+
+
+def op_rmsnorm_rope(buf_ptr, ld, rows, D, eps, gain, rope=False, grid=(0, 0, 0), split=(44, 42, 42),
+                    theta=10000.0, stream=None):
+    _check(lib().wan_op_rmsnorm_rope(buf_ptr, ld, rows, D, eps, _ptr(gain), int(rope), grid[0], grid[1], grid[2],
+                                     split[0], split[1], split[2], theta, _stream(stream)), "wan_op_rmsnorm_rope")
+
+
+def op_patchify(latent, X, stream=None):
+    B, Cc, F, Hz, Wz = latent.shape
+    _check(lib().wan_op_patchify(_ptr(latent), _dtype_code(latent), B, Cc, F, Hz, Wz, _ptr(X), _stream(stream)),
+           "wan_op_patchify")
+
+
+def op_unpatchify(rows, vel, stream=None):
+    B, Cc, F, Hz, Wz = vel.shape
+    _check(lib().wan_op_unpatchify(_ptr(rows), B, Cc, F, Hz, Wz, _ptr(vel), _stream(stream)), "wan_op_unpatchify")
+
+
+def op_sync(stream=None):
+    _check(lib().wan_op_sync(_stream(stream)), "wan_op_sync")
+
+
+def op_set_wait_limit_ns(ns: int):
+    lib().wan_op_set_wait_limit_ns(int(ns))

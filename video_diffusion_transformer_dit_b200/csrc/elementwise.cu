@@ -1,0 +1,399 @@
+// Bandwidth-bound kernels of the Wan DiT forward: LayerNorm with adaLN
+// modulation or affine, RMSNorm across heads with the 3-axis RoPE rotation,
+// the patchify gather, the unpatchify scatter (op-level), the small timestep
+// MLP GEMVs and dtype conversion.  One warp per row, 16-byte vector accesses
+// (8 bf16 per lane per step), fp32 statistics.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace wan {
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y; v[4] = c.x; v[5] = c.y; v[6] = d.x; v[7] = d.y;
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
+    uint4 u = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+    *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void load8f(const float* p, float (&v)[8]) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// ------------------------------------------------------------------ LayerNorm
+// mode 0: y = LN(x) * (1 + scale0 + scale1[m]) + shift0 + shift1[m]
+// mode 1: y = LN(x) * gamma + beta
+template <int NCH>
+__global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y,
+                                                        int rows, float eps, int mode, const float* gamma,
+                                                        const float* beta, const float* shift0, const float* shift1,
+                                                        const float* scale0, const float* scale1, int mod_div,
+                                                        long long mod_ld) {
+    constexpr int D = NCH * 256;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= rows) return;
+    const __nv_bfloat16* xr = x + (long long)row * D;
+    float v[NCH][8];
+    float s = 0.f;
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) {
+        load8(xr + (t * 32 + lane) * 8, v[t]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s += v[t][i];
+    }
+    const float mean = warp_sum(s) * (1.0f / D);
+    float ss = 0.f;
+#pragma unroll
+    for (int t = 0; t < NCH; ++t)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float d = v[t][i] - mean;
+            ss += d * d;
+        }
+    const float rstd = rsqrtf(warp_sum(ss) * (1.0f / D) + eps);
+    const long long m = (long long)(row / mod_div) * mod_ld;
+    __nv_bfloat16* yr = y + (long long)row * D;
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) {
+        const int c = (t * 32 + lane) * 8;
+        float a[8], bb[8], o[8];
+        if (mode == 0) {
+            float s1[8], h1[8];
+            load8f(scale0 + c, a);
+            load8f(shift0 + c, bb);
+            load8f(scale1 + m + c, s1);
+            load8f(shift1 + m + c, h1);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = (v[t][i] - mean) * rstd * (1.0f + a[i] + s1[i]) + (bb[i] + h1[i]);
+        } else {
+            load8f(gamma + c, a);
+            load8f(beta + c, bb);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = (v[t][i] - mean) * rstd * a[i] + bb[i];
+        }
+        store8(yr + c, o);
+    }
+}
+
+cudaError_t launch_layernorm(const void* x, void* y, int rows, int D, float eps, int mode, const float* gamma,
+                             const float* beta, const float* shift0, const float* shift1, const float* scale0,
+                             const float* scale1, int mod_div, long long mod_ld, const LaunchCtx& ctx) {
+    if (rows <= 0) return cudaSuccess;
+    if (D % 256) return cudaErrorInvalidValue;
+    if (mod_div <= 0) mod_div = 1;
+    dim3 grid((rows + 7) / 8);
+    auto X = reinterpret_cast<const __nv_bfloat16*>(x);
+    auto Y = reinterpret_cast<__nv_bfloat16*>(y);
+#define WAN_LN_CASE(n)                                                                                             \
+    case n:                                                                                                        \
+        layernorm_kernel<n><<<grid, 256, 0, ctx.stream>>>(X, Y, rows, eps, mode, gamma, beta, shift0, shift1, scale0, \
+                                                          scale1, mod_div, mod_ld);                                \
+        break;
+    switch (D / 256) {
+        WAN_LN_CASE(1) WAN_LN_CASE(2) WAN_LN_CASE(3) WAN_LN_CASE(4) WAN_LN_CASE(6) WAN_LN_CASE(8) WAN_LN_CASE(12)
+        WAN_LN_CASE(16) WAN_LN_CASE(20) WAN_LN_CASE(24)
+        default: return cudaErrorInvalidValue;
+    }
+#undef WAN_LN_CASE
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ RMSNorm across heads + RoPE
+// Pair p (0..63) of a 128-wide head: axis t for p < nt, h for p < nt + nh, else w.
+__device__ __forceinline__ float2 rope_cs(const RopeTables& rt, int p, int f, int i, int j) {
+    if (p < rt.nt) return __ldg(rt.t + f * rt.nt + p);
+    p -= rt.nt;
+    if (p < rt.nh) return __ldg(rt.h + i * rt.nh + p);
+    p -= rt.nh;
+    return __ldg(rt.w + j * rt.nw + p);
+}
+
+template <int NCH>
+__global__ void __launch_bounds__(256) rmsnorm_rope_kernel(__nv_bfloat16* buf, long long ld, int rows, float eps,
+                                                           const float* gains, long long gain_stride,
+                                                           long long seg_stride, RopeTables rt, int use_rope,
+                                                           int rope_L) {
+    constexpr int D = NCH * 256;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= rows) return;
+    const int seg = blockIdx.y;
+    __nv_bfloat16* xr = buf + (long long)row * ld + seg * seg_stride;
+    const float* g = gains + seg * gain_stride;
+    float v[NCH][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) {
+        load8(xr + (t * 32 + lane) * 8, v[t]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss += v[t][i] * v[t][i];
+    }
+    const float rs = rsqrtf(warp_sum(ss) * (1.0f / D) + eps);
+    int f = 0, ii = 0, jj = 0;
+    if (use_rope) {
+        const int l = row % rope_L;
+        const int hw = rt.Hp * rt.Wp;
+        f = l / hw;
+        const int rem = l - f * hw;
+        ii = rem / rt.Wp;
+        jj = rem - ii * rt.Wp;
+    }
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) {
+        const int c = (t * 32 + lane) * 8;
+        float gg[8], o[8];
+        load8f(g + c, gg);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = v[t][i] * rs * gg[i];
+        if (use_rope) {
+            const int p0 = (c & 127) >> 1;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 cs = rope_cs(rt, p0 + k, f, ii, jj);
+                const float a = o[2 * k], b = o[2 * k + 1];
+                o[2 * k] = a * cs.x - b * cs.y;
+                o[2 * k + 1] = a * cs.y + b * cs.x;
+            }
+        }
+        store8(xr + c, o);
+    }
+}
+
+cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float eps, const float* gains,
+                                long long gain_stride, int nseg, long long seg_stride, const RopeTables* rope,
+                                int rope_L, const LaunchCtx& ctx) {
+    if (rows <= 0 || nseg <= 0) return cudaSuccess;
+    if (D % 256 || ld % 8 || seg_stride % 8) return cudaErrorInvalidValue;
+    RopeTables rt{};
+    int use_rope = 0;
+    if (rope) {
+        rt = *rope;
+        use_rope = 1;
+        if (rope_L <= 0) return cudaErrorInvalidValue;
+    } else {
+        rope_L = 1;
+    }
+    dim3 grid((rows + 7) / 8, nseg);
+    auto Bp = reinterpret_cast<__nv_bfloat16*>(buf);
+#define WAN_RMS_CASE(n)                                                                                           \
+    case n:                                                                                                       \
+        rmsnorm_rope_kernel<n><<<grid, 256, 0, ctx.stream>>>(Bp, ld, rows, eps, gains, gain_stride, seg_stride, rt, \
+                                                             use_rope, rope_L);                                   \
+        break;
+    switch (D / 256) {
+        WAN_RMS_CASE(1) WAN_RMS_CASE(2) WAN_RMS_CASE(3) WAN_RMS_CASE(4) WAN_RMS_CASE(6) WAN_RMS_CASE(8)
+        WAN_RMS_CASE(12) WAN_RMS_CASE(16) WAN_RMS_CASE(20) WAN_RMS_CASE(24)
+        default: return cudaErrorInvalidValue;
+    }
+#undef WAN_RMS_CASE
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ patchify / unpatchify
+// X[b * L + (f * Hp + i) * Wp + j, c * 4 + kh * 2 + kw] = latent[b, c, f, 2i + kh, 2j + kw]
+template <typename T>
+__global__ void patchify_kernel(const T* __restrict__ lat, __nv_bfloat16* __restrict__ X, int B, int C, int F, int Hz,
+                                int Wz) {
+    const int Hp = Hz >> 1, Wp = Wz >> 1;
+    const long long L = (long long)F * Hp * Wp;
+    const long long total = (long long)B * L * C;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int c = idx % C;
+        const long long row = idx / C;
+        const int b = row / L;
+        const long long l = row - (long long)b * L;
+        const int f = l / (Hp * Wp);
+        const int rem = l - (long long)f * (Hp * Wp);
+        const int i = rem / Wp, j = rem - (rem / Wp) * Wp;
+        const T* src = lat + ((((long long)b * C + c) * F + f) * Hz + 2 * i) * Wz + 2 * j;
+        float a = (float)src[0], bb = (float)src[1], cc = (float)src[Wz], d = (float)src[Wz + 1];
+        uint2 u = make_uint2(pack_bf16(a, bb), pack_bf16(cc, d));
+        *reinterpret_cast<uint2*>(X + row * (4 * C) + 4 * c) = u;
+    }
+}
+
+cudaError_t launch_patchify(const void* latent, int latent_dtype, int B, int C, int F, int Hz, int Wz, void* X,
+                            const LaunchCtx& ctx) {
+    const long long total = (long long)B * F * (Hz / 2) * (Wz / 2) * C;
+    if (total <= 0) return cudaSuccess;
+    int grid = (int)((total + 255) / 256);
+    if (grid > ctx.num_sms * 16) grid = ctx.num_sms * 16;
+    if (latent_dtype == 0)
+        patchify_kernel<float><<<grid, 256, 0, ctx.stream>>>(reinterpret_cast<const float*>(latent),
+                                                              reinterpret_cast<__nv_bfloat16*>(X), B, C, F, Hz, Wz);
+    else
+        patchify_kernel<__nv_bfloat16><<<grid, 256, 0, ctx.stream>>>(reinterpret_cast<const __nv_bfloat16*>(latent),
+                                                                      reinterpret_cast<__nv_bfloat16*>(X), B, C, F, Hz,
+                                                                      Wz);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// vel[b, ch, f, 2i + kh, 2j + kw] = rows[b * L + token, (kh * 2 + kw) * C + ch]
+__global__ void unpatchify_kernel(const float* __restrict__ rows, float* __restrict__ vel, int B, int C, int F, int Hz,
+                                  int Wz) {
+    const int Hp = Hz >> 1, Wp = Wz >> 1;
+    const long long L = (long long)F * Hp * Wp;
+    const long long total = (long long)B * L * 4 * C;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int col = idx % (4 * C);
+        const long long row = idx / (4 * C);
+        const int b = row / L;
+        const long long l = row - (long long)b * L;
+        const int f = l / (Hp * Wp);
+        const int rem = l - (long long)f * (Hp * Wp);
+        const int i = rem / Wp, j = rem - (rem / Wp) * Wp;
+        const int ch = col % C, s = col / C, kh = s >> 1, kw = s & 1;
+        vel[((((long long)b * C + ch) * F + f) * Hz + 2 * i + kh) * Wz + 2 * j + kw] = rows[idx];
+    }
+}
+
+cudaError_t launch_unpatchify(const float* rows, int B, int C, int F, int Hz, int Wz, float* vel,
+                              const LaunchCtx& ctx) {
+    const long long total = (long long)B * F * (Hz / 2) * (Wz / 2) * 4 * C;
+    if (total <= 0) return cudaSuccess;
+    int grid = (int)((total + 255) / 256);
+    if (grid > ctx.num_sms * 16) grid = ctx.num_sms * 16;
+    unpatchify_kernel<<<grid, 256, 0, ctx.stream>>>(rows, vel, B, C, F, Hz, Wz);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ small GEMV (timestep MLP)
+// One warp per output column n, all B rows of x at once (B <= 8).
+__global__ void __launch_bounds__(256) gemv_kernel(const __nv_bfloat16* __restrict__ W, const float* __restrict__ bias,
+                                                   const float* __restrict__ x, long long ldx, float* __restrict__ out,
+                                                   long long ldout, int B, int N, int K, int act_in, int act_out) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = blockIdx.x * 8 + warp;
+    if (n >= N) return;
+    float acc[8];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[b] = 0.f;
+    const __nv_bfloat16* w = W + (long long)n * K;
+    const int half = K / 2;
+    for (int k0 = lane * 8; k0 < K; k0 += 256) {
+        float wv[8];
+        load8(w + k0, wv);
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            if (b >= B) break;
+            float xv[8];
+            if (act_in == 2) {
+                // timestep sinusoid: [cos(t w_k), sin(t w_k)], w_k = 1e4^(-k / half), computed in double
+                const double t = (double)x[b * ldx];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int k = k0 + i;
+                    const int kk = k < half ? k : k - half;
+                    const double w_k = exp(-9.210340371976184 * (double)kk / (double)half);  // ln(1e4)
+                    xv[i] = (float)(k < half ? cos(t * w_k) : sin(t * w_k));
+                }
+            } else {
+                load8f(x + b * ldx + k0, xv);
+                if (act_in == 1) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) xv[i] = xv[i] / (1.0f + __expf(-xv[i]));
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[b] = fmaf(wv[i], xv[i], acc[b]);
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+        if (b >= B) break;
+        float s = warp_sum(acc[b]);
+        if (lane == 0) {
+            s += bias ? bias[n] : 0.f;
+            if (act_out == 1) s = s / (1.0f + __expf(-s));
+            out[b * ldout + n] = s;
+        }
+    }
+}
+
+cudaError_t launch_gemv(const void* W, const float* bias, const float* x, long long ldx, float* out, long long ldout,
+                        int B, int N, int K, int act_in, int act_out, const LaunchCtx& ctx) {
+    if (B <= 0 || N <= 0) return cudaSuccess;
+    if (B > 8 || K % 8) return cudaErrorInvalidValue;
+    gemv_kernel<<<(N + 7) / 8, 256, 0, ctx.stream>>>(reinterpret_cast<const __nv_bfloat16*>(W), bias, x, ldx, out,
+                                                      ldout, B, N, K, act_in, act_out);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ per-token timestep features
+__global__ void sinusoid_kernel(const float* __restrict__ t, long long n, int dim, __nv_bfloat16* __restrict__ out) {
+    const int half = dim / 2;
+    const long long total = n * dim;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const long long r = idx / dim;
+        const int k = idx - r * dim;
+        const int kk = k < half ? k : k - half;
+        const double w_k = exp(-9.210340371976184 * (double)kk / (double)half);  // ln(1e4)
+        const double a = (double)t[r] * w_k;
+        out[idx] = __float2bfloat16_rn((float)(k < half ? cos(a) : sin(a)));
+    }
+}
+
+cudaError_t launch_sinusoid_bf16(const float* t, long long n, int dim, void* out, const LaunchCtx& ctx) {
+    if (n <= 0) return cudaSuccess;
+    long long g = (n * dim + 255) / 256;
+    if (g > ctx.num_sms * 16) g = ctx.num_sms * 16;
+    sinusoid_kernel<<<(int)g, 256, 0, ctx.stream>>>(t, n, dim, reinterpret_cast<__nv_bfloat16*>(out));
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+__global__ void silu_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ out, long long n) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const float v = x[i];
+        out[i] = __float2bfloat16_rn(v / (1.0f + __expf(-v)));
+    }
+}
+
+cudaError_t launch_silu_bf16(const float* x, void* out, long long n, const LaunchCtx& ctx) {
+    if (n <= 0) return cudaSuccess;
+    long long g = (n + 255) / 256;
+    if (g > ctx.num_sms * 16) g = ctx.num_sms * 16;
+    silu_bf16_kernel<<<(int)g, 256, 0, ctx.stream>>>(x, reinterpret_cast<__nv_bfloat16*>(out), n);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ dtype conversion
+__global__ void convert_kernel(const void* src, int sd, void* dst, int dd, long long n) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        float v = sd == 0 ? reinterpret_cast<const float*>(src)[i]
+                          : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(src)[i]);
+        if (dd == 0)
+            reinterpret_cast<float*>(dst)[i] = v;
+        else
+            reinterpret_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(v);
+    }
+}
+
+cudaError_t launch_convert(const void* src, int src_dtype, void* dst, int dst_dtype, long long n,
+                           cudaStream_t stream) {
+    if (n <= 0) return cudaSuccess;
+    long long g = (n + 255) / 256;
+    if (g > 4096) g = 4096;
+    convert_kernel<<<(int)g, 256, 0, stream>>>(src, src_dtype, dst, dst_dtype, n);
+    return cudaGetLastError();
+}
+
+}  // namespace wan

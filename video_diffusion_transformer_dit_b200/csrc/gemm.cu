@@ -1,0 +1,363 @@
+// tcgen05 GEMM for every linear layer of the Wan DiT forward: C = epi(A . W^T)
+// with A [M, K] activations and W [N, K] nn.Linear weights, both bf16 and
+// K-major, fp32 accumulation in tensor memory.
+//
+// One persistent CTA per SM, 6 warps:
+//   warp 0      TMA producer: 128 x 64 A tile and BN x 64 W tile per stage,
+//               128-byte swizzle, STAGES-deep mbarrier ring;
+//   warp 1      tensor-memory owner and MMA issuer (one thread): 4 x
+//               tcgen05.mma (M=128, N=BN, K=16) per stage into one of two
+//               TMEM accumulators (2 x BN columns), commit frees the stage;
+//   warps 2..5  epilogue: tcgen05.ld of 32 rows x 32 columns per warp, fused
+//               bias / GELU-tanh / gate * residual / unpatchify scatter, while
+//               the MMA warp already accumulates the next tile in the other
+//               TMEM buffer.
+// Tiles are walked N-fastest (an A row block stays in L2 while its N tiles
+// run) unless W is the larger operand, then M-fastest.
+#include <cstdio>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace wan {
+
+struct GemmParams {
+    int M, N, K;
+    int num_m, num_n, num_tiles;
+    int m_fastest;
+    EpiParams epi;
+    WaitCtl wc;
+};
+
+template <int BN>
+struct GemmCfg {
+    static constexpr int BM = 128;
+    static constexpr int BK = 64;
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+};
+
+__device__ __forceinline__ void tile_coords(int tile, const GemmParams& p, int& mb, int& nb) {
+    if (p.m_fastest) {
+        mb = tile % p.num_m;
+        nb = tile / p.num_m;
+    } else {
+        nb = tile % p.num_n;
+        mb = tile / p.num_n;
+    }
+}
+
+// Epilogue of 32 consecutive columns [c, c + 32) of one row.
+__device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int c, const uint32_t (&r)[32]) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    if (e.bias) {
+        const float4* b4 = reinterpret_cast<const float4*>(e.bias + c);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float4 b = __ldg(b4 + i);
+            v[4 * i] += b.x;
+            v[4 * i + 1] += b.y;
+            v[4 * i + 2] += b.z;
+            v[4 * i + 3] += b.w;
+        }
+    }
+    switch (e.kind) {
+        case EPI_BIAS:
+        case EPI_BIAS_GELU:
+        case EPI_BIAS_SILU: {
+            if (e.kind == EPI_BIAS_GELU) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_f(v[i]);
+            } else if (e.kind == EPI_BIAS_SILU) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = v[i] / (1.0f + __expf(-v[i]));
+            }
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint4 u;
+                u.x = pack_bf16(v[8 * i], v[8 * i + 1]);
+                u.y = pack_bf16(v[8 * i + 2], v[8 * i + 3]);
+                u.z = pack_bf16(v[8 * i + 4], v[8 * i + 5]);
+                u.w = pack_bf16(v[8 * i + 6], v[8 * i + 7]);
+                dst[i] = u;
+            }
+            break;
+        }
+        case EPI_GATE_RESIDUAL:
+        case EPI_RESIDUAL: {
+            uint4* xp = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
+            const float* g1 = e.gate1 ? e.gate1 + (long long)(row / e.mod_div) * e.mod_ld + c : nullptr;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint4 xu = xp[i];
+                uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
+                uint32_t ow[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    float2 xf = unpack_bf16(xw[h]);
+                    const int cc = 8 * i + 2 * h;
+                    float a0 = v[cc], a1 = v[cc + 1];
+                    if (e.kind == EPI_GATE_RESIDUAL) {
+                        float g0 = e.gate0[c + cc] + (g1 ? g1[cc] : 0.0f);
+                        float gg = e.gate0[c + cc + 1] + (g1 ? g1[cc + 1] : 0.0f);
+                        ow[h] = pack_bf16(xf.x + a0 * g0, xf.y + a1 * gg);
+                    } else {
+                        float2 ab = unpack_bf16(pack_bf16(a0, a1));  // the branch output is bf16 first
+                        ow[h] = pack_bf16(xf.x + ab.x, xf.y + ab.y);
+                    }
+                }
+                xp[i] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            }
+            break;
+        }
+        case EPI_BIAS_F32: {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(e.out) + (long long)row * e.ldo + c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            break;
+        }
+        case EPI_UNPATCHIFY: {
+            // row = b * L + token, token = (f * Hp + i) * Wp + j; column = (kh * 2 + kw) * C + ch
+            const int Hp = e.Hz >> 1, Wp = e.Wz >> 1;
+            const int b = row / e.L;
+            const int l = row - b * e.L;
+            const int f = l / (Hp * Wp);
+            const int rem = l - f * (Hp * Wp);
+            const int ii = rem / Wp;
+            const int jj = rem - ii * Wp;
+            float* vel = reinterpret_cast<float*>(e.out);
+#pragma unroll 4
+            for (int t = 0; t < 32; ++t) {
+                const int col = c + t;
+                const int ch = col % e.C;
+                const int s = col / e.C;
+                const int kh = s >> 1, kw = s & 1;
+                const long long idx =
+                    ((((long long)b * e.C + ch) * e.F + f) * e.Hz + (2 * ii + kh)) * e.Wz + (2 * jj + kw);
+                vel[idx] = __bfloat162float(__float2bfloat16_rn(v[t]));
+            }
+            break;
+        }
+        default:
+            break;
+    }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p) {
+    using Cfg = GemmCfg<BN>;
+    constexpr int STAGES = Cfg::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull + a, 1);
+            mbar_init(tempty + a, 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int kblocks = p.K / Cfg::BK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t armed = 0, armed_par = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+                int mb, nb;
+                tile_coords(tile, p, mb, nb);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.wc)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(full + stage, Cfg::STAGE_BYTES);
+                    tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, full + stage, kb * Cfg::BK, mb * Cfg::BM);
+                    tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, full + stage, kb * Cfg::BK, nb * BN);
+                    armed |= 1u << stage;
+                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (!ok) {  // drain the loads still in flight before the CTA exits
+                for (int s = 0; s < STAGES; ++s)
+                    if (armed & (1u << s)) mbar_drain(full + s, (armed_par >> s) & 1u, 200000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            constexpr uint32_t IDESC = idesc_bf16(128, BN, false);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true, issued = false;
+            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+                if (!mbar_wait(tempty + acc, acc_phase ^ 1, abort_flag, p.wc)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(full + stage, phase, abort_flag, p.wc)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * Cfg::A_BYTES);
+                    const uint32_t b0 = smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < Cfg::BK / 16; ++k) {
+                        umma_bf16_ss(d_tmem, sdesc_kmajor_sw128(a0 + 32 * k), sdesc_kmajor_sw128(b0 + 32 * k), IDESC,
+                                     (kb | k) != 0);
+                    }
+                    issued = true;
+                    umma_commit(empty + stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(tfull + acc);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+            if (!ok && issued) {  // let the tensor core finish before TMEM is freed
+                umma_commit(drain);
+                mbar_drain(drain, 0, 200000000ull);
+            }
+        }
+    } else {
+        // ---------------- epilogue warps ----------------
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+            int mb, nb;
+            tile_coords(tile, p, mb, nb);
+            if (!mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc)) break;
+            tc_fence_after();
+            const int row = mb * 128 + q * 32 + lane;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(taddr + c0, r);
+                tmem_ld_wait(r);
+                if (row < p.M) epilogue_chunk(p.epi, row, nb * BN + c0, r);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty + acc);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+template <int BN>
+static cudaError_t set_gemm_attr() {
+    return cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                GemmCfg<BN>::SMEM_BYTES);
+}
+
+cudaError_t init_gemm_attributes() {
+    cudaError_t e = set_gemm_attr<256>();
+    if (e == cudaSuccess) e = set_gemm_attr<128>();
+    if (e == cudaSuccess) e = set_gemm_attr<64>();
+    return e;
+}
+
+template <int BN>
+static cudaError_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                                  const LaunchCtx& ctx) {
+    using Cfg = GemmCfg<BN>;
+    int grid = p.num_tiles < ctx.num_sms ? p.num_tiles : ctx.num_sms;
+    gemm_tc_kernel<BN><<<grid, 192, Cfg::SMEM_BYTES, ctx.stream>>>(ta, tb, p);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long ldw, int M, int N, int K,
+                        const EpiParams& epi, const LaunchCtx& ctx) {
+    if (M <= 0) return cudaSuccess;
+    if (K <= 0 || K % 64 != 0 || N <= 0 || N % 64 != 0 || lda % 8 != 0 || ldw % 8 != 0)
+        return cudaErrorInvalidValue;
+    if ((reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15)) return cudaErrorInvalidValue;
+    int BN = (N % 256 == 0) ? 256 : (N % 128 == 0) ? 128 : 64;
+    GemmParams p;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.num_m = (M + 127) / 128;
+    p.num_n = N / BN;
+    p.num_tiles = p.num_m * p.num_n;
+    // walk M fastest when the weight operand is the bigger one (few row blocks)
+    p.m_fastest = ((long long)M < (long long)N) ? 1 : 0;
+    p.epi = epi;
+    if (p.epi.mod_div <= 0) p.epi.mod_div = 1;
+    p.wc.err = ctx.err;
+    p.wc.limit_ns = ctx.wait_limit_ns;
+    CUtensorMap ta, tb;
+    if (!make_tmap_2d(&ta, A, K, M, lda, 64, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tb, W, K, N, ldw, 64, BN)) return cudaErrorInvalidValue;
+    switch (BN) {
+        case 256: return launch_gemm_bn<256>(ta, tb, p, ctx);
+        case 128: return launch_gemm_bn<128>(ta, tb, p, ctx);
+        default: return launch_gemm_bn<64>(ta, tb, p, ctx);
+    }
+}
+
+}  // namespace wan
