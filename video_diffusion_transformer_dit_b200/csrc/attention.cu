@@ -191,7 +191,8 @@ __global__ void __launch_bounds__(192, 1)
         bool ok = true;
         for (int j = 0; j < nk; ++j) {
             const int s = j & 1;
-            if (!mbar_wait(s_full + s, (j >> 1) & 1, abort_flag, p.wc)) { ok = false; break; }
+            // every tcgen05.ld/st below is warp-collective: keep the warp's decisions uniform
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, (j >> 1) & 1, abort_flag, p.wc))) { ok = false; break; }
             tc_fence_after();
             uint32_t sv[4][32];
 #pragma unroll
@@ -230,23 +231,24 @@ __global__ void __launch_bounds__(192, 1)
                 }
             // P buffer and O are free once P_{j-1} V_{j-1} has completed
             if (j > 0) {
-                if (!mbar_wait(o_done, (j - 1) & 1, abort_flag, p.wc)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag, p.wc))) { ok = false; break; }
                 tc_fence_after();
             }
-            if (rescale) {
-                const float alpha = ex2_approx(m_run - m_use);  // 0 on the first tile
-                if (j > 0) {
+            // alpha = 1 for rows that keep their maximum; 0 on the first tile
+            const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;
+            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t ov[32];
-                        tmem_ld32(TM_O + lane_off + c * 32, ov);
-                        tmem_ld_wait(ov);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(TM_O + lane_off + c * 32, ov);
+                    tmem_ld_wait(ov);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                        tmem_st32(TM_O + lane_off + c * 32, ov);
-                    }
-                    tmem_st_wait();
+                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                    tmem_st32(TM_O + lane_off + c * 32, ov);
                 }
+                tmem_st_wait();
+            }
+            if (rescale) {
                 l_run *= alpha;
                 m_run = m_use;
             }
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
         }
-        if (ok && mbar_wait(o_done, (nk - 1) & 1, abort_flag, p.wc)) {
+        if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, (nk - 1) & 1, abort_flag, p.wc))) {
             tc_fence_after();
             const float inv = 1.0f / l_run;
             const int row = q0 + r;
@@ -290,6 +292,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

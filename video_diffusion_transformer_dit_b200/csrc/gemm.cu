@@ -281,7 +281,8 @@ __global__ void __launch_bounds__(192, 1)
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
             int mb, nb;
             tile_coords(tile, p, mb, nb);
-            if (!mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc)) break;
+            // tcgen05.ld is warp-collective: the whole warp takes the same branch
+            if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc))) break;
             tc_fence_after();
             const int row = mb * 128 + q * 32 + lane;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
@@ -302,6 +303,7 @@ __global__ void __launch_bounds__(192, 1)
 
     __syncthreads();
     if (warp == 1) {
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
