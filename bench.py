@@ -264,6 +264,90 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+# ---------------------------------------------------------------- single-kernel mode
+KERNELS = ("self_attention", "cross_attention", "gemm_qkv", "gemm_o", "gemm_ffn_up", "gemm_ffn_down", "layernorm",
+           "rmsnorm_rope")
+
+
+def run_kernel(args):
+    """Time one kernel of the forward alone at the workload's shapes (synthetic
+    operands on the device), K timed launches between CUDA events."""
+    import torch
+    from video_diffusion_transformer_dit_b200 import binding as Bd
+    from video_diffusion_transformer_dit_b200 import build, configs
+    build.build()
+    w = configs.workload(args.workload)
+    cfg = w["cfg"]
+    B, Cc, F, Hz, Wz = w["latent"]
+    L, Lc, D, Fd, H = F * (Hz // 2) * (Wz // 2), w["text_len"], cfg["dim"], cfg["ffn_dim"], cfg["heads"]
+    R = B * L
+    dev = "cuda"
+    g = torch.Generator(device=dev).manual_seed(0)
+
+    def rnd(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=g, device=dev) * scale).to(torch.bfloat16)
+
+    k = args.kernel
+    if k in ("self_attention", "cross_attention"):
+        Lk = L if k == "self_attention" else Lc
+        qkv = rnd(R, 3 * D)
+        kv = rnd(B * Lk, 2 * D)
+        o = torch.empty(R, D, dtype=torch.bfloat16, device=dev)
+        if k == "self_attention":
+            base = qkv.data_ptr()
+            fn = lambda: Bd.op_attention_ptr(base, 3 * D, base + 2 * D, 3 * D, base + 4 * D, 3 * D, o.data_ptr(), D,
+                                             B, H, L, L)
+        else:
+            q = rnd(R, D)
+            fn = lambda: Bd.op_attention_ptr(q.data_ptr(), D, kv.data_ptr(), 2 * D, kv.data_ptr() + 2 * D, 2 * D,
+                                             o.data_ptr(), D, B, H, L, Lk)
+        work, unit = 4.0 * L * Lk * D * B, "TFLOP/s"
+    elif k.startswith("gemm"):
+        N, K_, epi = {"gemm_qkv": (3 * D, D, "bias"), "gemm_o": (D, D, "gate_residual"),
+                      "gemm_ffn_up": (Fd, D, "bias_gelu"), "gemm_ffn_down": (D, Fd, "gate_residual")}[k]
+        A = rnd(R, K_)
+        Wt = rnd(N, K_, scale=0.02)
+        bias = torch.zeros(N, device=dev)
+        out = rnd(R, N)
+        gate0 = torch.full((N,), 0.1, device=dev)
+        gate1 = torch.zeros(B, 6 * N, device=dev)
+        fn = lambda: Bd.op_gemm(A, Wt, epi, out, bias=bias, gate0=gate0, gate1=gate1, mod_div=L, mod_ld=6 * N)
+        work, unit = 2.0 * R * N * K_, "TFLOP/s"
+    elif k == "layernorm":
+        x = rnd(R, D)
+        y = torch.empty_like(x)
+        sst = torch.zeros(6, D, device=dev)
+        tp = torch.zeros(B, 6 * D, device=dev)
+        fn = lambda: Bd.op_layernorm(x, y, 1e-6, 0, shift0=sst[0], shift1=tp, scale0=sst[1], scale1=tp,
+                                     mod_div=L, mod_ld=6 * D)
+        work, unit = 2.0 * R * D * 2, "GB/s"
+    elif k == "rmsnorm_rope":
+        qkv = rnd(R, 3 * D)
+        gain = torch.ones(D, device=dev)
+        fn = lambda: Bd.op_rmsnorm_rope(qkv.data_ptr(), 3 * D, R, D, 1e-6, gain, rope=True,
+                                        grid=(F, Hz // 2, Wz // 2))
+        work, unit = 2.0 * R * D * 2, "GB/s"
+    else:
+        raise SystemExit(f"unknown kernel {k}; one of {KERNELS}")
+    for _ in range(args.warmup):
+        fn()
+    Bd.op_sync()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    Bd.op_sync()
+    ms = e0.elapsed_time(e1) / args.steps
+    rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    peaks = load_peaks()
+    peak = peaks["bf16_tflops"] if unit == "TFLOP/s" else peaks["hbm_gbs"]
+    print(json.dumps({"kernel": k, "workload": args.workload, "avg_ms": ms, "achieved": rate, "unit": unit,
+                      "peak": peak, "frac": rate / peak, "peak_source": peaks["source"] + " (burst)",
+                      "work_per_launch": work, "launches": args.steps}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -273,7 +357,11 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=KERNELS, default=None,
+                    help="time one kernel alone at the workload's shapes (profiling aid)")
     args = ap.parse_args()
+    if args.kernel:
+        return run_kernel(args)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

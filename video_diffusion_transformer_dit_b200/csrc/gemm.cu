@@ -51,7 +51,8 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmParams& p, int& 
     }
 }
 
-// Epilogue of 32 consecutive columns [c, c + 32) of one row.
+// Epilogue of 32 consecutive columns [c, c + 32) of one row (KIND fixed at compile time).
+template <int KIND>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int c, const uint32_t (&r)[32]) {
     float v[32];
 #pragma unroll
@@ -67,14 +68,14 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
             v[4 * i + 3] += b.w;
         }
     }
-    switch (e.kind) {
+    switch (KIND) {
         case EPI_BIAS:
         case EPI_BIAS_GELU:
         case EPI_BIAS_SILU: {
-            if (e.kind == EPI_BIAS_GELU) {
+            if (KIND == EPI_BIAS_GELU) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_f(v[i]);
-            } else if (e.kind == EPI_BIAS_SILU) {
+            } else if (KIND == EPI_BIAS_SILU) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = v[i] / (1.0f + __expf(-v[i]));
             }
@@ -92,24 +93,47 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
         }
         case EPI_GATE_RESIDUAL:
         case EPI_RESIDUAL: {
+            // issue every load of the chunk before any store: x (4 x 16 B) and the gate rows
             uint4* xp = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
-            const float* g1 = e.gate1 ? e.gate1 + (long long)(row / e.mod_div) * e.mod_ld + c : nullptr;
+            uint4 xu[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xu[i] = xp[i];
+            float g[32];
+            if (KIND == EPI_GATE_RESIDUAL) {
+                const float4* g0 = reinterpret_cast<const float4*>(e.gate0 + c);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 a = __ldg(g0 + i);
+                    g[4 * i] = a.x;
+                    g[4 * i + 1] = a.y;
+                    g[4 * i + 2] = a.z;
+                    g[4 * i + 3] = a.w;
+                }
+                if (e.gate1) {
+                    const float4* g1 =
+                        reinterpret_cast<const float4*>(e.gate1 + (long long)(row / e.mod_div) * e.mod_ld + c);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 a = __ldg(g1 + i);
+                        g[4 * i] += a.x;
+                        g[4 * i + 1] += a.y;
+                        g[4 * i + 2] += a.z;
+                        g[4 * i + 3] += a.w;
+                    }
+                }
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                uint4 xu = xp[i];
-                uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
+                const uint32_t xw[4] = {xu[i].x, xu[i].y, xu[i].z, xu[i].w};
                 uint32_t ow[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    float2 xf = unpack_bf16(xw[h]);
+                    const float2 xf = unpack_bf16(xw[h]);
                     const int cc = 8 * i + 2 * h;
-                    float a0 = v[cc], a1 = v[cc + 1];
-                    if (e.kind == EPI_GATE_RESIDUAL) {
-                        float g0 = e.gate0[c + cc] + (g1 ? g1[cc] : 0.0f);
-                        float gg = e.gate0[c + cc + 1] + (g1 ? g1[cc + 1] : 0.0f);
-                        ow[h] = pack_bf16(xf.x + a0 * g0, xf.y + a1 * gg);
+                    if (KIND == EPI_GATE_RESIDUAL) {
+                        ow[h] = pack_bf16(xf.x + v[cc] * g[cc], xf.y + v[cc + 1] * g[cc + 1]);
                     } else {
-                        float2 ab = unpack_bf16(pack_bf16(a0, a1));  // the branch output is bf16 first
+                        const float2 ab = unpack_bf16(pack_bf16(v[cc], v[cc + 1]));  // the branch output is bf16 first
                         ow[h] = pack_bf16(xf.x + ab.x, xf.y + ab.y);
                     }
                 }
@@ -133,7 +157,7 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
             const int ii = rem / Wp;
             const int jj = rem - ii * Wp;
             float* vel = reinterpret_cast<float*>(e.out);
-#pragma unroll 4
+#pragma unroll
             for (int t = 0; t < 32; ++t) {
                 const int col = c + t;
                 const int ch = col % e.C;
@@ -150,7 +174,7 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
     }
 }
 
-template <int BN>
+template <int BN, int KIND>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
@@ -291,7 +315,7 @@ __global__ void __launch_bounds__(192, 1)
                 uint32_t r[32];
                 tmem_ld32(taddr + c0, r);
                 tmem_ld_wait(r);
-                if (row < p.M) epilogue_chunk(p.epi, row, nb * BN + c0, r);
+                if (row < p.M) epilogue_chunk<KIND>(p.epi, row, nb * BN + c0, r);
             }
             tc_fence_before();
             __syncwarp();
@@ -309,10 +333,22 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
+template <int BN, int KIND>
+static cudaError_t set_gemm_attr_one() {
+    return cudaFuncSetAttribute(gemm_tc_kernel<BN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                GemmCfg<BN>::SMEM_BYTES);
+}
+
 template <int BN>
 static cudaError_t set_gemm_attr() {
-    return cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                GemmCfg<BN>::SMEM_BYTES);
+    cudaError_t e = set_gemm_attr_one<BN, EPI_BIAS>();
+    if (e == cudaSuccess) e = set_gemm_attr_one<BN, EPI_BIAS_GELU>();
+    if (e == cudaSuccess) e = set_gemm_attr_one<BN, EPI_GATE_RESIDUAL>();
+    if (e == cudaSuccess) e = set_gemm_attr_one<BN, EPI_RESIDUAL>();
+    if (e == cudaSuccess) e = set_gemm_attr_one<BN, EPI_BIAS_F32>();
+    if (e == cudaSuccess) e = set_gemm_attr_one<BN, EPI_UNPATCHIFY>();
+    if (e == cudaSuccess) e = set_gemm_attr_one<BN, EPI_BIAS_SILU>();
+    return e;
 }
 
 cudaError_t init_gemm_attributes() {
@@ -326,8 +362,23 @@ template <int BN>
 static cudaError_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                                   const LaunchCtx& ctx) {
     using Cfg = GemmCfg<BN>;
-    int grid = p.num_tiles < ctx.num_sms ? p.num_tiles : ctx.num_sms;
-    gemm_tc_kernel<BN><<<grid, 192, Cfg::SMEM_BYTES, ctx.stream>>>(ta, tb, p);
+    const int grid = p.num_tiles < ctx.num_sms ? p.num_tiles : ctx.num_sms;
+    switch (p.epi.kind) {
+#define WAN_GEMM_CASE(K)                                                                   \
+    case K:                                                                                \
+        gemm_tc_kernel<BN, K><<<grid, 192, Cfg::SMEM_BYTES, ctx.stream>>>(ta, tb, p);     \
+        break;
+        WAN_GEMM_CASE(EPI_BIAS)
+        WAN_GEMM_CASE(EPI_BIAS_GELU)
+        WAN_GEMM_CASE(EPI_GATE_RESIDUAL)
+        WAN_GEMM_CASE(EPI_RESIDUAL)
+        WAN_GEMM_CASE(EPI_BIAS_F32)
+        WAN_GEMM_CASE(EPI_UNPATCHIFY)
+        WAN_GEMM_CASE(EPI_BIAS_SILU)
+#undef WAN_GEMM_CASE
+        default:
+            return cudaErrorInvalidValue;
+    }
     if (ctx.launches) ++*ctx.launches;
     return cudaGetLastError();
 }

@@ -57,9 +57,10 @@ struct KTimer {
         }
         return cudaSuccess;
     }
-    void begin(cudaStream_t s) { cudaEventRecord(ev[2 * n], s); }
+    // External records become event nodes when the forward is captured into a graph.
+    void begin(cudaStream_t s) { cudaEventRecordWithFlags(ev[2 * n], s, cudaEventRecordExternal); }
     void end(cudaStream_t s, int kc) {
-        cudaEventRecord(ev[2 * n + 1], s);
+        cudaEventRecordWithFlags(ev[2 * n + 1], s, cudaEventRecordExternal);
         if ((int)cls.size() <= n) cls.push_back(kc); else cls[n] = kc;
         ++n;
     }
