@@ -3,21 +3,24 @@
 // Used for the self-attention over the L video tokens and the
 // cross-attention to the Lc text tokens (ragged key tail masked).
 //
-// One CTA per (128-query tile, head, batch), 6 warps:
-//   warp 0      TMA producer: the Q tile once, then K and V tiles of 128 keys
-//               in two-slot rings (3-D tensor maps, rows past the sequence
-//               read as zero);
-//   warp 1      tensor-memory owner and MMA issuer: S_j = Q K_j^T into one of
-//               two 128-column TMEM buffers, issued one tile ahead, and
-//               O += P_j V_j into a third 128-column TMEM accumulator with V
-//               as an MN-major operand;
-//   warps 2..5  softmax, one query row per thread: tcgen05.ld of its S row,
-//               running max / sum in fp32 (log2 domain, exp2), the new
-//               probabilities written as bf16 into a swizzled shared tile P
-//               for the next MMA.  O is rescaled in TMEM only when the row
-//               maximum grows by more than 2^8 (the stale maximum is exact
-//               because the final division uses the same running sum); the
-//               last step divides by the sum and stores bf16 rows.
+// One CTA per (256 queries = two 128-row tiles, head, batch), 10 warps:
+//   warp 0      TMA producer: both Q tiles once, then K and V tiles of 128
+//               keys in two-slot rings (3-D tensor maps: rows past the
+//               sequence read as zero);
+//   warp 1      tensor-memory owner and MMA issuer.  Tensor memory holds
+//               S0 | S1 | O0 | O1 (4 x 128 fp32 columns).  Per key tile j it
+//               issues  PV0(j-1) S0(j) PV1(j-1) S1(j)  in that order, so the
+//               commit that publishes S_t(j) also covers PV_t(j-1);
+//   warps 2..5  softmax of tile 0, warps 6..9 softmax of tile 1 (one query
+//               row per thread, the two groups ping-pong with the tensor
+//               core): tcgen05.ld of the S row, running max / sum in fp32
+//               (log2 domain), probabilities packed to bf16 and written back
+//               with tcgen05.st over the S columns they came from (P aliases
+//               S), read there by the P.V MMA as its A operand.  O is
+//               rescaled in TMEM only when a row maximum grows by more than
+//               2^8 (the stale maximum is exact because the final division
+//               uses the same running sum); at the end each row is divided by
+//               its sum and stored as bf16.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -34,16 +37,18 @@ struct AttnParams {
 namespace attn {
 constexpr int TILE_BYTES = 128 * 128 * 2;  // one 128 x 128 bf16 tile = two 64-column swizzled halves
 constexpr int HALF_BYTES = 128 * 128;      // 128 rows x 128 bytes
-constexpr int SQ = 0;
-constexpr int SK = SQ + TILE_BYTES;          // 2 slots
-constexpr int SV = SK + 2 * TILE_BYTES;      // 2 slots
-constexpr int SP = SV + 2 * TILE_BYTES;      // 1 tile
-constexpr int SBAR = SP + TILE_BYTES;
+constexpr int KSTAGES = 2;
+constexpr int VSTAGES = 2;
+constexpr int SQ = 0;                              // Q0 | Q1
+constexpr int SK = SQ + 2 * TILE_BYTES;            // K ring
+constexpr int SV = SK + KSTAGES * TILE_BYTES;      // V ring
+constexpr int SBAR = SV + VSTAGES * TILE_BYTES;
 constexpr int SMEM_BYTES = SBAR + 256 + 1024;
-constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units
+constexpr int THREADS = 320;
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 }  // namespace attn
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(attn::THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
     using namespace attn;
@@ -51,36 +56,38 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SBAR);
     uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;   // [2]
-    uint64_t* k_empty = bars + 3;  // [2]
-    uint64_t* v_full = bars + 5;   // [2]
-    uint64_t* v_empty = bars + 7;  // [2]
-    uint64_t* s_full = bars + 9;   // [2]
-    uint64_t* s_empty = bars + 11; // [2]
-    uint64_t* p_full = bars + 13;
-    uint64_t* o_done = bars + 14;
-    uint64_t* drain = bars + 15;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    uint64_t* k_full = bars + 1;                 // [KSTAGES]
+    uint64_t* k_empty = k_full + KSTAGES;        // [KSTAGES]
+    uint64_t* v_full = k_empty + KSTAGES;        // [VSTAGES]
+    uint64_t* v_empty = v_full + VSTAGES;        // [VSTAGES]
+    uint64_t* s_full = v_empty + VSTAGES;        // [2] per query tile
+    uint64_t* p_full = s_full + 2;               // [2]
+    uint64_t* o_final = p_full + 2;              // [2]
+    uint64_t* drain = o_final + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int q0 = qt * 128;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int q0 = blockIdx.x * 256;
     const int nk = (p.Lk + 127) / 128;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < KSTAGES; ++s) {
             mbar_init(k_full + s, 1);
             mbar_init(k_empty + s, 1);
+        }
+        for (int s = 0; s < VSTAGES; ++s) {
             mbar_init(v_full + s, 1);
             mbar_init(v_empty + s, 1);
-            mbar_init(s_full + s, 1);
-            mbar_init(s_empty + s, 4);
         }
-        mbar_init(p_full, 4);
-        mbar_init(o_done, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(s_full + t, 1);
+            mbar_init(p_full + t, 4);
+            mbar_init(o_final + t, 1);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -96,39 +103,39 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t TM_S0 = tmem, TM_O = tmem + 256;
 
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- producer ----------------
-            uint32_t armed = 0, armed_par = 0;  // bits: q=0, k slots 1..2, v slots 3..4
+            uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
             bool ok = true;
-            mbar_expect_tx(q_full, TILE_BYTES);
-            tma_load_3d(smem + SQ, &tmQ, q_full, h * 128, q0, b);
-            tma_load_3d(smem + SQ + HALF_BYTES, &tmQ, q_full, h * 128 + 64, q0, b);
-            armed |= 1u;
-            for (int j = 0; ok && j < nk; ++j) {
-                const int s = j & 1;
-                const uint32_t par = (j >> 1) & 1;
-                if (!mbar_wait(k_empty + s, par ^ 1, abort_flag, p.wc)) { ok = false; break; }
-                mbar_expect_tx(k_full + s, TILE_BYTES);
-                tma_load_3d(smem + SK + s * TILE_BYTES, &tmK, k_full + s, h * 128, j * 128, b);
-                tma_load_3d(smem + SK + s * TILE_BYTES + HALF_BYTES, &tmK, k_full + s, h * 128 + 64, j * 128, b);
-                armed |= 2u << s;
-                armed_par = (armed_par & ~(2u << s)) | (par << (1 + s));
-                if (!mbar_wait(v_empty + s, par ^ 1, abort_flag, p.wc)) { ok = false; break; }
-                mbar_expect_tx(v_full + s, TILE_BYTES);
-                tma_load_3d(smem + SV + s * TILE_BYTES, &tmV, v_full + s, h * 128, j * 128, b);
-                tma_load_3d(smem + SV + s * TILE_BYTES + HALF_BYTES, &tmV, v_full + s, h * 128 + 64, j * 128, b);
-                armed |= 8u << s;
-                armed_par = (armed_par & ~(8u << s)) | (par << (3 + s));
+            mbar_expect_tx(q_full, 2 * TILE_BYTES);
+            for (int t = 0; t < 2; ++t) {
+                tma_load_3d(smem + SQ + t * TILE_BYTES, &tmQ, q_full, h * 128, q0 + 128 * t, b);
+                tma_load_3d(smem + SQ + t * TILE_BYTES + HALF_BYTES, &tmQ, q_full, h * 128 + 64, q0 + 128 * t, b);
             }
-            if (!ok) {
+            for (int j = 0; ok && j < nk; ++j) {
+                const int ks = j % KSTAGES, vs = j % VSTAGES;
+                const uint32_t kp = (j / KSTAGES) & 1, vp = (j / VSTAGES) & 1;
+                if (!mbar_wait(k_empty + ks, kp ^ 1, abort_flag, p.wc)) { ok = false; break; }
+                mbar_expect_tx(k_full + ks, TILE_BYTES);
+                tma_load_3d(smem + SK + ks * TILE_BYTES, &tmK, k_full + ks, h * 128, j * 128, b);
+                tma_load_3d(smem + SK + ks * TILE_BYTES + HALF_BYTES, &tmK, k_full + ks, h * 128 + 64, j * 128, b);
+                karmed |= 1u << ks;
+                kpar = (kpar & ~(1u << ks)) | (kp << ks);
+                if (!mbar_wait(v_empty + vs, vp ^ 1, abort_flag, p.wc)) { ok = false; break; }
+                mbar_expect_tx(v_full + vs, TILE_BYTES);
+                tma_load_3d(smem + SV + vs * TILE_BYTES, &tmV, v_full + vs, h * 128, j * 128, b);
+                tma_load_3d(smem + SV + vs * TILE_BYTES + HALF_BYTES, &tmV, v_full + vs, h * 128 + 64, j * 128, b);
+                varmed |= 1u << vs;
+                vpar = (vpar & ~(1u << vs)) | (vp << vs);
+            }
+            if (!ok) {  // drain the loads still in flight before the CTA exits
                 mbar_drain(q_full, 0, 200000000ull);
-                for (int s = 0; s < 2; ++s) {
-                    if (armed & (2u << s)) mbar_drain(k_full + s, (armed_par >> (1 + s)) & 1, 200000000ull);
-                    if (armed & (8u << s)) mbar_drain(v_full + s, (armed_par >> (3 + s)) & 1, 200000000ull);
-                }
+                for (int s = 0; s < KSTAGES; ++s)
+                    if (karmed & (1u << s)) mbar_drain(k_full + s, (kpar >> s) & 1, 200000000ull);
+                for (int s = 0; s < VSTAGES; ++s)
+                    if (varmed & (1u << s)) mbar_drain(v_full + s, (vpar >> s) & 1, 200000000ull);
             }
         }
     } else if (warp == 1) {
@@ -137,143 +144,143 @@ __global__ void __launch_bounds__(192, 1)
             constexpr uint32_t ID_QK = idesc_bf16(128, 128, false);
             constexpr uint32_t ID_PV = idesc_bf16(128, 128, true);
             const uint32_t sq = smem_u32(smem + SQ);
-            const uint32_t sp = smem_u32(smem + SP);
             bool ok = mbar_wait(q_full, 0, abort_flag, p.wc);
             bool issued = false;
-            auto issue_s = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!mbar_wait(k_full + s, (j >> 1) & 1, abort_flag, p.wc)) return false;
-                if (j >= 2 && !mbar_wait(s_empty + s, ((j - 2) >> 1) & 1, abort_flag, p.wc)) return false;
+            // S_t(j) = Q_t K_j^T into TMEM columns [128 t, 128 t + 128)
+            auto issue_s = [&](int t, int j) -> bool {
+                const int ks = j % KSTAGES;
+                if (t == 0 && !mbar_wait(k_full + ks, (j / KSTAGES) & 1, abort_flag, p.wc)) return false;
                 tc_fence_after();
-                const uint32_t sk = smem_u32(smem + SK + s * TILE_BYTES);
+                const uint32_t sk = smem_u32(smem + SK + ks * TILE_BYTES);
+                const uint32_t sqt = sq + t * TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-                    umma_bf16_ss(TM_S0 + s * 128, sdesc_kmajor_sw128(sq + off), sdesc_kmajor_sw128(sk + off), ID_QK,
+                    umma_bf16_ss(tmem + t * 128, sdesc_kmajor_sw128(sqt + off), sdesc_kmajor_sw128(sk + off), ID_QK,
                                  kk != 0);
                 }
                 issued = true;
-                umma_commit(s_full + s);
-                umma_commit(k_empty + s);
+                umma_commit(s_full + t);
+                if (t == 1) umma_commit(k_empty + ks);
                 return true;
             };
-            if (ok) ok = issue_s(0);
-            for (int j = 0; ok && j < nk; ++j) {
-                if (j + 1 < nk && !issue_s(j + 1)) { ok = false; break; }
-                const int s = j & 1;
-                if (!mbar_wait(p_full, j & 1, abort_flag, p.wc)) { ok = false; break; }
-                if (!mbar_wait(v_full + s, (j >> 1) & 1, abort_flag, p.wc)) { ok = false; break; }
+            // O_t += P_t(j) V_j, P_t read from the S_t columns (bf16 pairs)
+            auto issue_pv = [&](int t, int j) -> bool {
+                const int vs = j % VSTAGES;
+                if (!mbar_wait(p_full + t, j & 1, abort_flag, p.wc)) return false;
+                if (t == 0 && !mbar_wait(v_full + vs, (j / VSTAGES) & 1, abort_flag, p.wc)) return false;
                 tc_fence_after();
-                const uint32_t sv = smem_u32(smem + SV + s * TILE_BYTES);
+                const uint32_t sv = smem_u32(smem + SV + vs * TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    // P: K-major over keys; V: rows are keys, 64-wide d halves HALF_BYTES apart
-                    const uint32_t poff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-                    umma_bf16_ss(TM_O, sdesc_kmajor_sw128(sp + poff), sdesc_mnmajor_sw128(sv + kk * 2048, HALF_BYTES),
-                                 ID_PV, (j | kk) != 0);
+                    umma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                                 sdesc_mnmajor_sw128(sv + kk * 2048, HALF_BYTES), ID_PV, (j | kk) != 0);
                 }
-                umma_commit(v_empty + s);
-                umma_commit(o_done);
+                if (t == 1) umma_commit(v_empty + vs);
+                if (j == nk - 1) umma_commit(o_final + t);
+                return true;
+            };
+            if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
+            for (int j = 0; ok && j < nk; ++j) {
+                if (!issue_pv(0, j)) { ok = false; break; }
+                if (j + 1 < nk && !issue_s(0, j + 1)) { ok = false; break; }
+                if (!issue_pv(1, j)) { ok = false; break; }
+                if (j + 1 < nk && !issue_s(1, j + 1)) { ok = false; break; }
             }
-            if (!ok && issued) {
+            if (!ok && issued) {  // let the tensor core finish before TMEM is freed
                 umma_commit(drain);
                 mbar_drain(drain, 0, 200000000ull);
             }
         }
     } else {
         // ---------------- softmax / output warps ----------------
-        const int qq = warp & 3;
-        const int r = qq * 32 + lane;                     // row inside the tile == TMEM lane
+        const int t = (warp - 2) >> 2;                   // query tile 0 or 1
+        const int qq = warp & 3;                         // TMEM lane quarter
+        const int r = qq * 32 + lane;                    // row inside the tile == TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(qq * 32) << 16;
-        uint8_t* prow = smem + SP + r * 128;
-        const int sw = r & 7;
+        const uint32_t TS = tmem + t * 128 + lane_off;   // S_t (and P_t)
+        const uint32_t TO = tmem + 256 + t * 128 + lane_off;
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         for (int j = 0; j < nk; ++j) {
-            const int s = j & 1;
-            // every tcgen05.ld/st below is warp-collective: keep the warp's decisions uniform
-            if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, (j >> 1) & 1, abort_flag, p.wc))) { ok = false; break; }
+            // all tcgen05.ld/st below are warp-collective: the warp's decisions stay uniform
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full + t, j & 1, abort_flag, p.wc))) { ok = false; break; }
             tc_fence_after();
             uint32_t sv[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(TM_S0 + lane_off + s * 128 + c * 32, sv[c]);
+            for (int c = 0; c < 4; ++c) tmem_ld32(TS + c * 32, sv[c]);
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_empty + s);
 
             const int valid = min(128, p.Lk - j * 128);
-            float mx = -INFINITY;
+            if (valid < 128) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    float x = __uint_as_float(sv[c][i]);
-                    if (c * 32 + i >= valid) x = -INFINITY;
-                    sv[c][i] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
-                }
-            const float m_tile = mx * p.scale_log2;
+                    for (int i = 0; i < 32; ++i)
+                        if (c * 32 + i >= valid) sv[c][i] = __float_as_uint(-INFINITY);
+            }
+            // row maximum: independent 3-input max chains
+            float mx[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float a = __uint_as_float(sv[c][0]);
+                const float bb = __uint_as_float(sv[c][1]);
+#pragma unroll
+                for (int i = 2; i < 32; i += 2) a = max3f(a, __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
+                mx[c] = fmaxf(a, bb);
+            }
+            const float m_tile = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3])) * p.scale_log2;
             const float m_new = fmaxf(m_run, m_tile);
             const bool rescale = m_new > m_run + RESCALE_THRESHOLD;
             const float m_use = rescale ? m_new : m_run;
-            float rowsum = 0.0f;
+            // probabilities, packed to bf16 pairs; four independent partial sums
             uint32_t pk[64];
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     const float e0 = ex2_approx(fmaf(__uint_as_float(sv[c][i]), p.scale_log2, -m_use));
                     const float e1 = ex2_approx(fmaf(__uint_as_float(sv[c][i + 1]), p.scale_log2, -m_use));
-                    rowsum += e0 + e1;
+                    ps[c] += e0 + e1;
                     pk[c * 16 + i / 2] = pack_bf16(e0, e1);
                 }
-            // P buffer and O are free once P_{j-1} V_{j-1} has completed
-            if (j > 0) {
-                if (!__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag, p.wc))) { ok = false; break; }
-                tc_fence_after();
-            }
-            // alpha = 1 for rows that keep their maximum; 0 on the first tile
-            const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;
+            // O_t is idle here: the commit of S_t(j) also covered P_t(j-1) V_{j-1}
+            const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;  // 0 on the first tile
             if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t ov[32];
-                    tmem_ld32(TM_O + lane_off + c * 32, ov);
+                    tmem_ld32(TO + c * 32, ov);
                     tmem_ld_wait(ov);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st32(TM_O + lane_off + c * 32, ov);
+                    tmem_st32(TO + c * 32, ov);
                 }
-                tmem_st_wait();
             }
+            // P_t over the first 64 columns of S_t
+            tmem_st32(TS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_st32(TS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+            tmem_st_wait();
             if (rescale) {
                 l_run *= alpha;
                 m_run = m_use;
             }
-            l_run += rowsum;
-            // P row -> shared memory, K-major with the 128-byte swizzle
-#pragma unroll
-            for (int ch = 0; ch < 16; ++ch) {
-                const int half = ch >> 3, c16 = ch & 7;
-                uint4 u = make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-                *reinterpret_cast<uint4*>(prow + half * HALF_BYTES + ((c16 ^ sw) << 4)) = u;
-            }
-            fence_proxy_async_smem();
+            l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(p_full + t);
         }
-        if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, (nk - 1) & 1, abort_flag, p.wc))) {
+        if (ok && __all_sync(0xffffffffu, mbar_wait(o_final + t, 0, abort_flag, p.wc))) {
             tc_fence_after();
             const float inv = 1.0f / l_run;
-            const int row = q0 + r;
+            const int row = q0 + 128 * t + r;
             __nv_bfloat16* orow = p.o + ((long long)b * p.Lq + row) * p.ldo + h * 128;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t ov[32];
-                tmem_ld32(TM_O + lane_off + c * 32, ov);
+                tmem_ld32(TO + c * 32, ov);
                 tmem_ld_wait(ov);
                 if (row < p.Lq) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
@@ -328,8 +335,8 @@ cudaError_t launch_attention(const void* q, long long ldq, const void* k, long l
     p.scale_log2 = 1.4426950408889634f / sqrtf(128.0f);
     p.wc.err = ctx.err;
     p.wc.limit_ns = ctx.wait_limit_ns;
-    dim3 grid((Lq + 127) / 128, heads, B);
-    attn_tc_kernel<<<grid, 192, attn::SMEM_BYTES, ctx.stream>>>(tq, tk, tv, p);
+    dim3 grid((Lq + 255) / 256, heads, B);
+    attn_tc_kernel<<<grid, attn::THREADS, attn::SMEM_BYTES, ctx.stream>>>(tq, tk, tv, p);
     if (ctx.launches) ++*ctx.launches;
     return cudaGetLastError();
 }
