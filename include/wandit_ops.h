@@ -89,6 +89,30 @@ WANDIT_API wan_status wan_op_rmsnorm_rope(void* buf, int64_t ld, int rows, int D
                                int rope, int Fp, int Hp, int Wp, int rope_t, int rope_h, int rope_w,
                                float theta, void* stream);
 
+/* Allocation-free variant of wan_op_rmsnorm_rope (same arguments, same
+ * result).  The pages have no counterpart: this exists for callers that must
+ * not allocate device memory while they run -- serving stacks whose own pool
+ * allocator holds (nearly) all of HBM, so a library cudaMalloc fails or breaks
+ * their accounting, and latency-critical loops that cannot take the implicit
+ * synchronisation cudaMalloc / cudaFree may cause.  wan_op_rmsnorm_rope
+ * allocates its cos/sin table per call; this variant keeps it in a fixed
+ * __device__ array of 1024 positions x 64 pairs (512 KiB) that every GPU
+ * loading the library holds until the process exits, and calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *  - Limit: Fp, Hp and Wp (post-patch grid) must each be <= 1024, the
+ *    rope_max_seq_len of the Wan configs; larger grids return WAN_ESHAPE
+ *    before anything is launched.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address with cudaGetSymbolAddress and caches it; make
+ *    that first call before any stream capture on the device.
+ *  - Every call rewrites the part of the array it uses and all calls share
+ *    it: calls that can overlap on the GPU (different streams without an
+ *    ordering between them) race on the table and must be serialised.     */
+WANDIT_API wan_status wan_op_rmsnorm_rope_noalloc(void* buf, int64_t ld, int rows, int D, float eps,
+                                                  const float* gain, int rope, int Fp, int Hp, int Wp,
+                                                  int rope_t, int rope_h, int rope_w, float theta,
+                                                  void* stream);
+
 /* Patchify gather: latent [B, C, F, Hz, Wz] (f32 or bf16) -> X bf16
  * [B * L, C * 4] with token order (f, i, j) and feature order (c, kh, kw) --
  * the input view of patch_embedding = Conv3d(k = s = (1,2,2)).               */

@@ -30,7 +30,7 @@ SYMBOLS = ["wan_dit_create", "wan_dit_load_weights", "wan_dit_missing_weights", 
            "wan_dit_flops",
            "wan_dit_last_error", "wan_status_string", "wan_dit_destroy",
            "wan_op_gemm", "wan_op_attention", "wan_op_layernorm", "wan_op_rmsnorm_rope", "wan_op_patchify",
-           "wan_op_unpatchify", "wan_op_sync", "wan_op_set_wait_limit_ns"]
+           "wan_op_unpatchify", "wan_op_sync", "wan_op_set_wait_limit_ns", "wan_op_rmsnorm_rope_noalloc"]
 
 
 class WanError(RuntimeError):
@@ -86,6 +86,7 @@ def lib() -> C.CDLL:
         "wan_op_attention": (I, [P, I64, P, I64, P, I64, P, I64, I, I, I, I, P]),
         "wan_op_layernorm": (I, [P, P, I, I, F, I, P, P, P, P, P, P, I, I64, P]),
         "wan_op_rmsnorm_rope": (I, [P, I64, I, I, F, P, I, I, I, I, I, I, I, F, P]),
+        "wan_op_rmsnorm_rope_noalloc": (I, [P, I64, I, I, F, P, I, I, I, I, I, I, I, F, P]),
         "wan_op_patchify": (I, [P, I, I, I, I, I, I, P, P]),
         "wan_op_unpatchify": (I, [P, I, I, I, I, I, P, P]),
         "wan_op_sync": (I, [P]),
@@ -266,6 +267,14 @@ def op_rmsnorm_rope(buf_ptr, ld, rows, D, eps, gain, rope=False, grid=(0, 0, 0),
                     theta=10000.0, stream=None):
     _check(lib().wan_op_rmsnorm_rope(buf_ptr, ld, rows, D, eps, _ptr(gain), int(rope), grid[0], grid[1], grid[2],
                                      split[0], split[1], split[2], theta, _stream(stream)), "wan_op_rmsnorm_rope")
+
+
+def op_rmsnorm_rope_noalloc(buf_ptr, ld, rows, D, eps, gain, rope=True, grid=(0, 0, 0), split=(44, 42, 42),
+                            theta=10000.0, stream=None):
+    """wan_op_rmsnorm_rope without any device allocation (fixed 1024-position table)."""
+    _check(lib().wan_op_rmsnorm_rope_noalloc(buf_ptr, ld, rows, D, eps, _ptr(gain), int(rope), grid[0], grid[1],
+                                             grid[2], split[0], split[1], split[2], theta, _stream(stream)),
+           "wan_op_rmsnorm_rope_noalloc")
 
 
 def op_patchify(latent, X, stream=None):
