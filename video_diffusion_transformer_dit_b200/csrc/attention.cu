@@ -3,7 +3,9 @@
 // Used for the self-attention over the L video tokens and the
 // cross-attention to the Lc text tokens (ragged key tail masked).
 //
-// One CTA per (256 queries = two 128-row tiles, head, batch), 10 warps:
+// One CTA per (256 queries = two 128-row tiles, head, batch), 12 warps in
+// three warpgroups; the first gives registers to the two softmax groups
+// (56 / 224 / 224 per thread, 64512 in all = 384 threads x 168 at launch):
 //   warp 0      TMA producer: both Q tiles once, then K and V tiles of 128
 //               keys in two-slot rings (3-D tensor maps: rows past the
 //               sequence read as zero);
@@ -11,7 +13,8 @@
 //               S0 | S1 | O0 | O1 (4 x 128 fp32 columns).  Per key tile j it
 //               issues  PV0(j-1) S0(j) PV1(j-1) S1(j)  in that order, so the
 //               commit that publishes S_t(j) also covers PV_t(j-1);
-//   warps 2..5  softmax of tile 0, warps 6..9 softmax of tile 1 (one query
+//   warps 2..3  idle;
+//   warps 4..7  softmax of tile 0, warps 8..11 softmax of tile 1 (one query
 //               row per thread, the two groups ping-pong with the tensor
 //               core): tcgen05.ld of the S row, running max / sum in fp32
 //               (log2 domain), probabilities packed to bf16 and written back
@@ -44,7 +47,11 @@ constexpr int SK = SQ + 2 * TILE_BYTES;            // K ring
 constexpr int SV = SK + KSTAGES * TILE_BYTES;      // V ring
 constexpr int SBAR = SV + VSTAGES * TILE_BYTES;
 constexpr int SMEM_BYTES = SBAR + 256 + 1024;
-constexpr int THREADS = 320;
+constexpr int THREADS = 384;
+constexpr int REGS_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
+constexpr int REGS_CONTROL = 56;   // warpgroup 0: producer + MMA issuer
+constexpr int REGS_SOFTMAX = 224;  // warpgroups 1, 2
+static_assert(128 * REGS_CONTROL + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH, "register split");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 }  // namespace attn
 
@@ -104,6 +111,8 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    if (warp < 4) {
+        regs_dealloc<REGS_CONTROL>();
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- producer ----------------
@@ -192,9 +201,11 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                 mbar_drain(drain, 0, 200000000ull);
             }
         }
+    }
     } else {
+        regs_alloc<REGS_SOFTMAX>();
         // ---------------- softmax / output warps ----------------
-        const int t = (warp - 2) >> 2;                   // query tile 0 or 1
+        const int t = (warp - 4) >> 2;                   // query tile 0 or 1
         const int qq = warp & 3;                         // TMEM lane quarter
         const int r = qq * 32 + lane;                    // row inside the tile == TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(qq * 32) << 16;
