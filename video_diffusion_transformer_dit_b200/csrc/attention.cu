@@ -40,7 +40,10 @@ struct AttnParams {
 namespace attn {
 constexpr int TILE_BYTES = 128 * 128 * 2;  // one 128 x 128 bf16 tile = two 64-column swizzled halves
 constexpr int HALF_BYTES = 128 * 128;      // 128 rows x 128 bytes
-constexpr int KSTAGES = 2;
+#ifndef WAN_ATTN_KSTAGES
+#define WAN_ATTN_KSTAGES 2
+#endif
+constexpr int KSTAGES = WAN_ATTN_KSTAGES;
 constexpr int VSTAGES = 2;
 constexpr int SQ = 0;                              // Q0 | Q1
 constexpr int SK = SQ + 2 * TILE_BYTES;            // K ring
@@ -49,10 +52,18 @@ constexpr int SBAR = SV + VSTAGES * TILE_BYTES;
 constexpr int SMEM_BYTES = SBAR + 256 + 1024;
 constexpr int THREADS = 384;
 constexpr int REGS_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
-constexpr int REGS_CONTROL = 56;   // warpgroup 0: producer + MMA issuer
-constexpr int REGS_SOFTMAX = 224;  // warpgroups 1, 2
+#ifndef WAN_ATTN_REGS_CONTROL
+#define WAN_ATTN_REGS_CONTROL 56
+#define WAN_ATTN_REGS_SOFTMAX 224
+#endif
+constexpr int REGS_CONTROL = WAN_ATTN_REGS_CONTROL;  // warpgroup 0: producer + MMA issuer
+constexpr int REGS_SOFTMAX = WAN_ATTN_REGS_SOFTMAX;  // warpgroups 1, 2
 static_assert(128 * REGS_CONTROL + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH, "register split");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+#ifndef WAN_ATTN_EMU_PAIRS
+#define WAN_ATTN_EMU_PAIRS 2
+#endif
+constexpr int EMU_PAIRS_OF_8 = WAN_ATTN_EMU_PAIRS;  // column pairs per 8 on the software exp2
 }  // namespace attn
 
 __global__ void __launch_bounds__(attn::THREADS, 1)
@@ -231,32 +242,50 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     for (int i = 0; i < 32; ++i)
                         if (c * 32 + i >= valid) sv[c][i] = __float_as_uint(-INFINITY);
             }
-            // row maximum: independent 3-input max chains
-            float mx[4];
+            // row maximum: eight independent 3-input max chains
+            float mx[8];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float a = __uint_as_float(sv[c][0]);
-                const float bb = __uint_as_float(sv[c][1]);
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t* v = &sv[q >> 1][(q & 1) * 16];
+                float a = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
 #pragma unroll
-                for (int i = 2; i < 32; i += 2) a = max3f(a, __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
-                mx[c] = fmaxf(a, bb);
+                for (int i = 2; i < 16; i += 2) a = max3f(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+                mx[q] = a;
             }
-            const float m_tile = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3])) * p.scale_log2;
+            const float m_tile =
+                max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * p.scale_log2;
             const float m_new = fmaxf(m_run, m_tile);
             const bool rescale = m_new > m_run + RESCALE_THRESHOLD;
             const float m_use = rescale ? m_new : m_run;
-            // probabilities, packed to bf16 pairs; four independent partial sums
-            uint32_t pk[64];
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            // probabilities on packed fp32 pairs, EMU_PAIRS_OF_8 of every 8 pairs on the
+            // software exp2 (FMA pipe); each 32-column chunk is packed to bf16 and
+            // stored over its own S columns (P_t = first 64 columns of S_t) at once
+            uint64_t ps2[2] = {0ull, 0ull};
+            const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
+            const uint64_t negm2 = f2pack(-m_use, -m_use);
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pc[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
-                    const float e0 = ex2_approx(fmaf(__uint_as_float(sv[c][i]), p.scale_log2, -m_use));
-                    const float e1 = ex2_approx(fmaf(__uint_as_float(sv[c][i + 1]), p.scale_log2, -m_use));
-                    ps[c] += e0 + e1;
-                    pk[c * 16 + i / 2] = pack_bf16(e0, e1);
+                    const uint64_t x2 = fma2(f2pack(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])), scale2, negm2);
+                    float e0, e1;
+                    if (((i >> 1) & 7) >= 8 - EMU_PAIRS_OF_8) {
+                        ex2_poly2(x2, e0, e1);
+                    } else {
+                        float x0, x1;
+                        f2unpack(x2, x0, x1);
+                        e0 = ex2_approx(x0);
+                        e1 = ex2_approx(x1);
+                    }
+                    ps2[(i >> 1) & 1] = add2(ps2[(i >> 1) & 1], f2pack(e0, e1));
+                    pc[i / 2] = pack_bf16(e0, e1);
                 }
+                tmem_st16(TS + c * 16, pc);
+            }
+            float ps[4];
+            f2unpack(ps2[0], ps[0], ps[1]);
+            f2unpack(ps2[1], ps[2], ps[3]);
             // O_t is idle here: the commit of S_t(j) also covered P_t(j-1) V_{j-1}
             const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;  // 0 on the first tile
             if (j > 0 && __any_sync(0xffffffffu, rescale)) {
@@ -270,9 +299,6 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     tmem_st32(TO + c * 32, ov);
                 }
             }
-            // P_t over the first 64 columns of S_t
-            tmem_st32(TS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(TS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_st_wait();
             if (rescale) {
                 l_run *= alpha;

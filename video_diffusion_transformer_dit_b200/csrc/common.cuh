@@ -213,6 +213,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         WAN_IN32(r)
         : "memory");
 }
+#define WAN_IN16(r)                                                                                             \
+    "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), \
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        WAN_IN16(r)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
@@ -276,6 +286,54 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
     return y;
 }
+// Packed fp32 pairs (two lanes of one 64-bit register) for the f32x2 ALU ops.
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for a pair of x <= 8 on the FMA and integer pipes instead of the MUFU:
+// x = n + f with n the nearest integer (magic-number rounding) and |f| <= 1/2,
+// p(f) ~ 2^f from a cubic fitted by weighted least squares on Chebyshev nodes
+// (coefficients from gen_exp2_poly.py, relative error < 8e-5), then n added to
+// the exponent field.  x is clamped at -125 so the exponent never underflows
+// (2^-125 ~ 2e-38 stands in for 0).
+__device__ __forceinline__ void ex2_poly2(uint64_t x2, float& e0, float& e1) {
+    float x0, x1;
+    f2unpack(x2, x0, x1);
+    const uint64_t xc = f2pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t magic = f2pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+    const uint64_t t2 = add2(xc, magic);
+    const uint64_t fr = sub2(xc, sub2(t2, magic));
+    uint64_t p2 = fma2(f2pack(5.508868396e-02f, 5.508868396e-02f), fr, f2pack(2.426040471e-01f, 2.426040471e-01f));
+    p2 = fma2(p2, fr, f2pack(6.932762265e-01f, 6.932762265e-01f));
+    p2 = fma2(p2, fr, f2pack(9.999289513e-01f, 9.999289513e-01f));
+    float p0, p1, t0, t1;
+    f2unpack(p2, p0, p1);
+    f2unpack(t2, t0, t1);
+    e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ float tanh_approx(float x) {
     float y;
     asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
