@@ -130,6 +130,23 @@ def cpu_sample(w, rows_small=128, rows_big=384, seed=0):
     return B * L / step_s, step_s, desc, sum(times)
 
 
+# ---------------------------------------------------------------- multi-rank plumbing
+def reduce_max(values, device):
+    """Max over ranks of per-rank timings (no-op in a single process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tokens_per_s(world, batch, tokens, ms_per_step):
+    """Every rank runs its own replica of the step: all ranks' tokens over the slowest rank's time."""
+    return world * batch * tokens / (ms_per_step * 1e-3)
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -217,10 +234,7 @@ def run_ours(args, rank, world, local_rank):
         ts_h[0].numel() * ts_h[0].element_size()
     d2h = vel_h.numel() * vel_h.element_size()
 
-    if world > 1:
-        t = torch.tensor([ms, ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_e2e = t.tolist()
+    ms, ms_e2e = reduce_max([ms, ms_e2e], dev)
 
     flops = dit.flops(B, F, Hz, Wz, Lc, int(w["timesteps"] == "per_token"))
     # dominant kernel: self-attention, 4 * L^2 * head_dim * heads * B flops per launch
@@ -231,7 +245,7 @@ def run_ours(args, rank, world, local_rank):
     peak = peaks["bf16_tflops_sustained"]
     result = {
         "metric": METRIC,
-        "value": world * B * L / (ms * 1e-3),
+        "value": whole_job_tokens_per_s(world, B, L, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -256,7 +270,7 @@ def run_ours(args, rank, world, local_rank):
                      "flops_per_launch": sa_flops, "avg_launch_ms": sa_avg_ms, "launches_per_step": sa_n,
                      "traffic": None},
         "kernel_ms_per_step": {c: v[0] for c, v in kt.items()},
-        "e2e": {"value": world * B * L / (ms_e2e * 1e-3), "unit": "tokens/s", "ms_per_step": ms_e2e,
+        "e2e": {"value": whole_job_tokens_per_s(world, B, L, ms_e2e), "unit": "tokens/s", "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches * args.steps,
         "clocks": clk,

@@ -125,6 +125,23 @@ WANDIT_API wan_status wan_op_patchify(const void* latent, int latent_dtype, int 
 WANDIT_API wan_status wan_op_unpatchify(const float* rows, int B, int C, int F, int Hz, int Wz,
                              float* velocity, void* stream);
 
+/* One flow-matching sampler step with classifier-free guidance
+ * ("【VLA与模仿学习】Wan2.1框架与训练源码导读" §7: CFG  v = v_uncond + s (v_cond - v_uncond),
+ * Euler update  x_next = x + (sigma_next - sigma) v; §6.1 x_sigma = (1 - sigma) z + sigma eps).
+ * x, v_cond, v_uncond, x_next: f32 device arrays of n elements, 16-byte aligned (x_next may
+ * alias x).  v_uncond == NULL means no guidance (v = v_cond).  With the CFG batch of
+ * wan_dit_forward (B = 2), v_cond / v_uncond are the two halves of its velocity output.   */
+WANDIT_API wan_status wan_op_cfg_euler(const float* x, const float* v_cond, const float* v_uncond,
+                                       float guidance, float sigma, float sigma_next, int64_t n,
+                                       float* x_next, void* stream);
+
+/* Self-test of the bounded on-chip waits every tcgen05 kernel uses: launches one
+ * warp that waits on an mbarrier nothing arrives on, with a time limit of
+ * `limit_ns` (clamped to [1 us, 1 s]).  The wait gives up, records the timeout in
+ * the op error word and the kernel returns; wan_op_sync() then reports
+ * WAN_ETIMEOUT and clears it.  Faults nothing and leaves the context usable.  */
+WANDIT_API wan_status wan_op_wait_selftest(int64_t limit_ns, void* stream);
+
 /* Synchronise `stream`; WAN_ETIMEOUT if an op kernel's bounded wait ran out
  * (flag cleared), WAN_ECUDA on a CUDA error.                                */
 WANDIT_API wan_status wan_op_sync(void* stream);

@@ -158,3 +158,42 @@ def test_abi_validation_and_missing_weights():
     assert e.value.name == "WAN_ESHAPE"
     v = dit.forward(lat.cuda(), t.cuda(), ctx.cuda(), sync=True)
     assert torch.isfinite(v).all()
+
+
+def _sampled_rows_case(cfg, shape, Lc, seed, per_token=False, n_rows=48):
+    from video_diffusion_transformer_dit_b200 import synth
+    B, Cc, F, Hz, Wz = shape
+    L = O.token_count(F, Hz, Wz)
+    W = synth.make_weights(cfg, seed=seed)
+    lat = synth.make_latent(shape, seed=seed)
+    ctx = synth.make_context(B, Lc, cfg["text_dim"], seed=seed)
+    t = synth.make_timestep_per_token(B, L, (Hz // 2) * (Wz // 2), seed=seed) if per_token else \
+        synth.make_timestep(B, 500.0)
+    dit = make_dit(cfg, B, L, Lc, W)
+    v = run_gpu(dit, lat, t, ctx)
+    dit.close()
+    g = torch.Generator().manual_seed(seed)
+    rows = torch.cat([torch.tensor([0, L - 1]), torch.randint(0, L, (n_rows,), generator=g)]).unique()
+    o = O.forward(lat.to(DT), t.to(DT), ctx.to(DT), to64(W), cfg, rows=rows)
+    idx = O.unpatch_index_map(Cc, F, Hz, Wz)[rows]
+    return rel_l2(v.reshape(B, -1)[:, idx], o), rows.numel()
+
+
+def test_forward_14b_widths_one_block_sampled_rows():
+    """Wan-14B widths (D 5120, 40 heads, FFN 13824, 512 text tokens), one block,
+    81-frame 720x1280 spatial grid on 3 latent frames (10800 tokens)."""
+    from video_diffusion_transformer_dit_b200 import configs
+    cfg = configs.model_config("wan2.1-14b", num_blocks=1)
+    err, n = _sampled_rows_case(cfg, (1, 16, 3, 90, 160), 512, seed=6)
+    print(f"\n14B widths one block, {n} sampled tokens rel-L2 {err:.3e}")
+    assert err < TOL
+
+
+def test_forward_5b_per_token_full_shape_one_block_sampled_rows():
+    """Wan2.2-5B shape at its full size (48 channels, 121 frames 704x1280 -> 27280
+    tokens, 512 text tokens) with per-token timesteps, one block."""
+    from video_diffusion_transformer_dit_b200 import configs
+    cfg = configs.model_config("wan2.2-5b", num_blocks=1)
+    err, n = _sampled_rows_case(cfg, (1, 48, 31, 44, 80), 512, seed=7, per_token=True)
+    print(f"\n5B full shape per-token one block, {n} sampled tokens rel-L2 {err:.3e}")
+    assert err < TOL

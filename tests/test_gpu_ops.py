@@ -243,3 +243,24 @@ def test_rmsnorm_rope(rope):
     got = d.cpu()
     assert rel_l2(got[:, D:2 * D], ref) < TOL
     assert torch.equal(got[:, :D], buf[:, :D]) and torch.equal(got[:, 2 * D:], buf[:, 2 * D:])
+
+
+# ------------------------------------------------------------------ sampler step (CFG + Euler)
+def test_cfg_euler_matches_oracle_and_worked_example():
+    g = torch.Generator().manual_seed(21)
+    shape = (1, 16, 21, 60, 104)
+    x, vc, vu = (torch.randn(*shape, generator=g) for _ in range(3))
+    out = torch.empty(shape, device="cuda")
+    B().op_cfg_euler(x.cuda(), vc.cuda(), vu.cuda(), 6.0, 0.75, 0.5, out)
+    B().op_sync()
+    ref = O.euler_step(x.to(DT), 0.75, 0.5, O.cfg_combine(vu.to(DT), vc.to(DT), 6.0))
+    assert rel_l2(out, ref) < 1e-6
+    # the hand-worked example of the flow-matching section: x=8, v=8, sigma 0.75 -> 0.5 -> 0
+    xs = torch.full((5,), 8.0, device="cuda")
+    vs = torch.full((5,), 8.0, device="cuda")
+    x1 = torch.empty_like(xs)
+    B().op_cfg_euler(xs, vs, None, 1.0, 0.75, 0.5, x1)
+    x2 = torch.empty_like(xs)
+    B().op_cfg_euler(x1, vs, None, 1.0, 0.5, 0.0, x2)
+    B().op_sync()
+    assert torch.equal(x1.cpu(), torch.full((5,), 6.0)) and torch.equal(x2.cpu(), torch.full((5,), 2.0))

@@ -30,7 +30,8 @@ SYMBOLS = ["wan_dit_create", "wan_dit_load_weights", "wan_dit_missing_weights", 
            "wan_dit_flops",
            "wan_dit_last_error", "wan_status_string", "wan_dit_destroy",
            "wan_op_gemm", "wan_op_attention", "wan_op_layernorm", "wan_op_rmsnorm_rope", "wan_op_patchify",
-           "wan_op_unpatchify", "wan_op_sync", "wan_op_set_wait_limit_ns", "wan_op_rmsnorm_rope_noalloc"]
+           "wan_op_unpatchify", "wan_op_sync", "wan_op_set_wait_limit_ns", "wan_op_rmsnorm_rope_noalloc", "wan_op_cfg_euler",
+           "wan_op_wait_selftest"]
 
 
 class WanError(RuntimeError):
@@ -90,6 +91,8 @@ def lib() -> C.CDLL:
         "wan_op_patchify": (I, [P, I, I, I, I, I, I, P, P]),
         "wan_op_unpatchify": (I, [P, I, I, I, I, I, P, P]),
         "wan_op_sync": (I, [P]),
+        "wan_op_cfg_euler": (I, [P, P, P, F, F, F, I64, P, P]),
+        "wan_op_wait_selftest": (I, [I64, P]),
         "wan_op_set_wait_limit_ns": (None, [I64]),
     }
     for name, (res, args) in sig.items():
@@ -286,6 +289,16 @@ def op_patchify(latent, X, stream=None):
 def op_unpatchify(rows, vel, stream=None):
     B, Cc, F, Hz, Wz = vel.shape
     _check(lib().wan_op_unpatchify(_ptr(rows), B, Cc, F, Hz, Wz, _ptr(vel), _stream(stream)), "wan_op_unpatchify")
+
+
+def op_cfg_euler(x, v_cond, v_uncond, guidance, sigma, sigma_next, out, stream=None):
+    """out = x + (sigma_next - sigma) * (v_uncond + guidance * (v_cond - v_uncond)); f32 CUDA tensors."""
+    _check(lib().wan_op_cfg_euler(_ptr(x), _ptr(v_cond), _ptr(v_uncond), guidance, sigma, sigma_next, x.numel(),
+                                  _ptr(out), _stream(stream)), "wan_op_cfg_euler")
+
+
+def op_wait_selftest(limit_ns, stream=None):
+    _check(lib().wan_op_wait_selftest(int(limit_ns), _stream(stream)), "wan_op_wait_selftest")
 
 
 def op_sync(stream=None):

@@ -87,7 +87,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
-        if (mbar_try_sleep(bar, parity, 100000u)) return true;
+        if (mbar_try_sleep(bar, parity, wc.limit_ns < 100000ull ? (uint32_t)wc.limit_ns : 100000u)) return true;
         if (*abort) return false;
         if (global_ns() - t0 > wc.limit_ns) {
             *abort = 1;

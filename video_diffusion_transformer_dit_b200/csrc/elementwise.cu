@@ -375,6 +375,66 @@ cudaError_t launch_silu_bf16(const float* x, void* out, long long n, const Launc
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ flow-matching sampler step
+// x_next = x + (sigma_next - sigma) * (v_u + s (v_c - v_u))   (v = v_c when v_u is null)
+__global__ void cfg_euler_kernel(const float* __restrict__ x, const float* __restrict__ vc,
+                                 const float* __restrict__ vu, float s, float dsigma, long long n,
+                                 float* __restrict__ xn) {
+    const long long n4 = n / 4;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += stride) {
+        const float4 a = reinterpret_cast<const float4*>(x)[i];
+        const float4 c = reinterpret_cast<const float4*>(vc)[i];
+        float4 v = c;
+        if (vu) {
+            const float4 u = reinterpret_cast<const float4*>(vu)[i];
+            v = make_float4(u.x + s * (c.x - u.x), u.y + s * (c.y - u.y), u.z + s * (c.z - u.z), u.w + s * (c.w - u.w));
+        }
+        reinterpret_cast<float4*>(xn)[i] =
+            make_float4(a.x + dsigma * v.x, a.y + dsigma * v.y, a.z + dsigma * v.z, a.w + dsigma * v.w);
+    }
+    for (long long i = n4 * 4 + blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += stride) {
+        const float v = vu ? vu[i] + s * (vc[i] - vu[i]) : vc[i];
+        xn[i] = x[i] + dsigma * v;
+    }
+}
+
+cudaError_t launch_cfg_euler(const float* x, const float* v_cond, const float* v_uncond, float guidance, float sigma,
+                             float sigma_next, long long n, float* x_next, const LaunchCtx& ctx) {
+    if (n <= 0) return cudaSuccess;
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(v_cond) |
+         reinterpret_cast<uintptr_t>(v_uncond) | reinterpret_cast<uintptr_t>(x_next)) & 15)
+        return cudaErrorInvalidValue;
+    long long g = (n / 4 + 255) / 256;
+    if (g < 1) g = 1;
+    if (g > ctx.num_sms * 8) g = ctx.num_sms * 8;
+    cfg_euler_kernel<<<(int)g, 256, 0, ctx.stream>>>(x, v_cond, v_uncond, guidance, sigma_next - sigma, n, x_next);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ bounded-wait self-test
+// One warp waits on an mbarrier that nothing ever arrives on; the bounded wait
+// gives up after limit_ns, raises the CTA's abort flag and records the timeout.
+__global__ void wait_selftest_kernel(int* err, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    WaitCtl wc{err, limit_ns};
+    mbar_wait(&bar, 0, &abort_flag, wc);
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, const LaunchCtx& ctx) {
+    wait_selftest_kernel<<<1, 32, 0, ctx.stream>>>(ctx.err, limit_ns);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ dtype conversion
 __global__ void convert_kernel(const void* src, int sd, void* dst, int dd, long long n) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {

@@ -95,6 +95,13 @@ cudaError_t launch_sinusoid_bf16(const float* t, long long n, int dim, void* out
 // out bf16 = SiLU(x f32), elementwise.
 cudaError_t launch_silu_bf16(const float* x, void* out, long long n, const LaunchCtx& ctx);
 
+// x_next = x + (sigma_next - sigma) * (v_uncond + guidance (v_cond - v_uncond)); v_uncond may be null.
+cudaError_t launch_cfg_euler(const float* x, const float* v_cond, const float* v_uncond, float guidance, float sigma,
+                             float sigma_next, long long n, float* x_next, const LaunchCtx& ctx);
+
+// One-warp kernel whose only mbarrier is never arrived on: exercises the bounded wait.
+cudaError_t launch_wait_selftest(uint64_t limit_ns, const LaunchCtx& ctx);
+
 // dst = convert(src), elementwise; dtypes 0 f32 / 1 bf16.
 cudaError_t launch_convert(const void* src, int src_dtype, void* dst, int dst_dtype, long long n,
                            cudaStream_t stream);

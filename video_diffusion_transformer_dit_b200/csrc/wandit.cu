@@ -924,6 +924,22 @@ wan_status wan_op_rmsnorm_rope(void* buf, int64_t ld, int rows, int D, float eps
     return op_status(e);
 }
 
+wan_status wan_op_wait_selftest(int64_t limit_ns, void* stream) {
+    LaunchCtx ctx;
+    if (!op_ctx(reinterpret_cast<cudaStream_t>(stream), &ctx)) return WAN_ECUDA;
+    const uint64_t lim = limit_ns < 1000 ? 1000ull : (limit_ns > 1000000000 ? 1000000000ull : (uint64_t)limit_ns);
+    return op_status(wan::launch_wait_selftest(lim, ctx));
+}
+
+wan_status wan_op_cfg_euler(const float* x, const float* v_cond, const float* v_uncond, float guidance, float sigma,
+                            float sigma_next, int64_t n, float* x_next, void* stream) {
+    if (!x || !v_cond || !x_next) return WAN_EINVAL;
+    if (n < 0) return WAN_ESHAPE;
+    LaunchCtx ctx;
+    if (!op_ctx(reinterpret_cast<cudaStream_t>(stream), &ctx)) return WAN_ECUDA;
+    return op_status(wan::launch_cfg_euler(x, v_cond, v_uncond, guidance, sigma, sigma_next, n, x_next, ctx));
+}
+
 wan_status wan_op_patchify(const void* latent, int latent_dtype, int B, int C, int F, int Hz, int Wz, void* X,
                            void* stream) {
     if (!latent || !X) return WAN_EINVAL;
