@@ -32,6 +32,18 @@ METRIC = "ms/denoise-step & tokens/s, Wan-1.3B-shape 480p; % of B200 bf16 TC pea
 DEFAULT_WORKLOAD = "wan1.3b-81f-480x832-cfg2"
 
 
+def measured_traffic(kernel, source):
+    """DRAM bytes per launch from the committed ncu capture, only while the kernel
+    source is unchanged since the capture (else None)."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "roofline_traffic.json")))[kernel]
+        sha = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()
+        return rec["dram_bytes_per_launch"] if sha == rec["source_sha256"] else None
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -268,7 +280,9 @@ def run_ours(args, rank, world, local_rank):
                      "peak": peak, "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None,
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
                      "flops_per_launch": sa_flops, "avg_launch_ms": sa_avg_ms, "launches_per_step": sa_n,
-                     "traffic": None},
+                     "traffic": measured_traffic("attn_tc_kernel",
+                                                 "video_diffusion_transformer_dit_b200/csrc/attention.cu"),
+                     "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
         "kernel_ms_per_step": {c: v[0] for c, v in kt.items()},
         "e2e": {"value": whole_job_tokens_per_s(world, B, L, ms_e2e), "unit": "tokens/s", "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
