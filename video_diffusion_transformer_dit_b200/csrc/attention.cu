@@ -63,6 +63,9 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 #ifndef WAN_ATTN_EMU_PAIRS
 #define WAN_ATTN_EMU_PAIRS 2
 #endif
+#ifndef WAN_ATTN_EX2_F32
+#define WAN_ATTN_EX2_F32 1   // 1: one ex2.approx.f32 per exponential; 0: ex2.approx.f16x2 pairs (measured slower)
+#endif
 constexpr int EMU_PAIRS_OF_8 = WAN_ATTN_EMU_PAIRS;  // column pairs per 8 on the software exp2
 }  // namespace attn
 
@@ -275,8 +278,12 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     } else {
                         float x0, x1;
                         f2unpack(x2, x0, x1);
+#if WAN_ATTN_EX2_F32
                         e0 = ex2_approx(x0);
                         e1 = ex2_approx(x1);
+#else
+                        ex2_f16x2(x0, x1, e0, e1);
+#endif
                     }
                     ps2[(i >> 1) & 1] = add2(ps2[(i >> 1) & 1], f2pack(e0, e1));
                     pc[i / 2] = pack_bf16(e0, e1);

@@ -306,6 +306,21 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
     return y;
 }
+// 2^x for a pair through one MUFU instruction: x rounded to f16 (relative error
+// of 2^x <= |x| 2^-11 ln 2, 0.13 % at |x| = 8), ex2.approx.f16x2, widened back
+// to fp32.  Two exponentials per MUFU issue instead of one.
+__device__ __forceinline__ void ex2_f16x2(float x0, float x1, float& e0, float& e1) {
+    uint32_t h, e;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x1), "f"(x0));  // x0 in the low half
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "cvt.f32.f16 %0, lo;\n\t"
+        "cvt.f32.f16 %1, hi;\n\t}"
+        : "=f"(e0), "=f"(e1)
+        : "r"(e));
+}
+
 // Packed fp32 pairs (two lanes of one 64-bit register) for the f32x2 ALU ops.
 __device__ __forceinline__ uint64_t f2pack(float a, float b) {
     uint64_t r;

@@ -2,13 +2,14 @@
 // with A [M, K] activations and W [N, K] nn.Linear weights, both bf16 and
 // K-major, fp32 accumulation in tensor memory.
 //
-// One persistent CTA per SM, 6 warps:
+// One persistent CTA per SM, 10 warps:
 //   warp 0      TMA producer: 128 x 64 A tile and BN x 64 W tile per stage,
 //               128-byte swizzle, STAGES-deep mbarrier ring;
 //   warp 1      tensor-memory owner and MMA issuer (one thread): 4 x
 //               tcgen05.mma (M=128, N=BN, K=16) per stage into one of two
 //               TMEM accumulators (2 x BN columns), commit frees the stage;
-//   warps 2..5  epilogue: tcgen05.ld of 32 rows x 32 columns per warp, fused
+//   warps 2..9  epilogue, two warps per TMEM lane quarter, each taking half of
+//               the tile's columns: tcgen05.ld of 32 rows x 32 columns, fused
 //               bias / GELU-tanh / gate * residual / unpatchify scatter, while
 //               the MMA warp already accumulates the next tile in the other
 //               TMEM buffer.
@@ -174,8 +175,11 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
     }
 }
 
+constexpr int EPI_WARPS = 8;
+constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
+
 template <int BN, int KIND>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
     using Cfg = GemmCfg<BN>;
@@ -202,7 +206,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull + a, 1);
-            mbar_init(tempty + a, 4);
+            mbar_init(tempty + a, EPI_WARPS);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -299,7 +303,9 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else {
         // ---------------- epilogue warps ----------------
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int q = warp & 3;                       // TMEM lane quarter this warp may access
+        const int chalf = (warp - 2) >> 2;            // which half of the tile's columns
+        constexpr int CW = BN / 2;                    // columns per epilogue warp
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
@@ -311,7 +317,7 @@ __global__ void __launch_bounds__(192, 1)
             const int row = mb * 128 + q * 32 + lane;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
+            for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
                 uint32_t r[32];
                 tmem_ld32(taddr + c0, r);
                 tmem_ld_wait(r);
@@ -366,7 +372,7 @@ static cudaError_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, 
     switch (p.epi.kind) {
 #define WAN_GEMM_CASE(K)                                                                   \
     case K:                                                                                \
-        gemm_tc_kernel<BN, K><<<grid, 192, Cfg::SMEM_BYTES, ctx.stream>>>(ta, tb, p);     \
+        gemm_tc_kernel<BN, K><<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, ctx.stream>>>(ta, tb, p); \
         break;
         WAN_GEMM_CASE(EPI_BIAS)
         WAN_GEMM_CASE(EPI_BIAS_GELU)
