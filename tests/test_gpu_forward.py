@@ -197,3 +197,24 @@ def test_forward_5b_per_token_full_shape_one_block_sampled_rows():
     err, n = _sampled_rows_case(cfg, (1, 48, 31, 44, 80), 512, seed=7, per_token=True)
     print(f"\n5B full shape per-token one block, {n} sampled tokens rel-L2 {err:.3e}")
     assert err < TOL
+
+
+def test_forward_33f_352x640_all_30_blocks_full_oracle():
+    """33 frames 352x640 (latent [1,16,9,44,80], 7920 tokens = 61 full 128-row
+    tiles + a ragged 112), all 30 blocks, every element against the full float64
+    oracle, with the per-block error report."""
+    cfg, W, lat, t, ctx = workload_inputs("wan1.3b-33f-352x640")
+    B, L, Lc = 1, O.token_count(*lat.shape[2:]), ctx.shape[1]
+    dit = make_dit(cfg, B, L, Lc, W)
+    dump = torch.zeros(cfg["num_blocks"] + 1, B * L, cfg["dim"], dtype=torch.bfloat16, device="cuda")
+    dit.set_block_dump(dump)
+    v = run_gpu(dit, lat, t, ctx)
+    dump = dump.cpu()
+    dit.close()
+    ref, blocks = O.forward(lat.to(DT), t.to(DT), ctx.to(DT), to64(W), cfg, return_blocks=True)
+    errs = [rel_l2(dump[i], blocks[i].reshape(B * L, -1)) for i in range(len(blocks))]
+    report("33f 352x640, 30 blocks", errs)
+    err = rel_l2(v, ref)
+    print(f"velocity rel-L2 {err:.3e}")
+    assert max(errs) < TOL
+    assert err < TOL
