@@ -31,6 +31,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 // ------------------------------------------------------------------ LayerNorm
 // mode 0: y = LN(x) * (1 + scale0 + scale1[m]) + shift0 + shift1[m]
 // mode 1: y = LN(x) * gamma + beta
+// mode 2: y = LN(x) * scale1[m] + shift1[m]   (modulation precombined, 1 + scale included)
 template <int NCH>
 __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y,
                                                         int rows, float eps, int mode, const float* gamma,
@@ -66,7 +67,12 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __r
     for (int t = 0; t < NCH; ++t) {
         const int c = (t * 32 + lane) * 8;
         float a[8], bb[8], o[8];
-        if (mode == 0) {
+        if (mode == 2) {
+            load8f(scale1 + m + c, a);
+            load8f(shift1 + m + c, bb);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = (v[t][i] - mean) * rstd * a[i] + bb[i];
+        } else if (mode == 0) {
             float s1[8], h1[8];
             load8f(scale0 + c, a);
             load8f(shift0 + c, bb);
@@ -104,6 +110,34 @@ cudaError_t launch_layernorm(const void* x, void* y, int rows, int D, float eps,
         default: return cudaErrorInvalidValue;
     }
 #undef WAN_LN_CASE
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ per-sample modulation, all blocks
+// out[n][b][k][c] = sst[n][k][c] + tproj[b][k][c] + (k == 1 || k == 4 ? 1 : 0)
+// (k: shift, scale, gate, c_shift, c_scale, c_gate; the "1 +" of the two scales folded in)
+__global__ void mod_combine_kernel(const float* __restrict__ sst, const float* __restrict__ tproj, float* __restrict__ out,
+                                   int N, int B, int D) {
+    const long long total = (long long)N * B * 6 * D;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+        const int c = i % D;
+        const long long r = i / D;
+        const int k = r % 6;
+        const long long nb = r / 6;
+        const int b = nb % B;
+        const int n = nb / B;
+        out[i] = sst[((long long)n * 6 + k) * D + c] + tproj[((long long)b * 6 + k) * D + c] + ((k == 1 || k == 4) ? 1.0f : 0.0f);
+    }
+}
+
+cudaError_t launch_mod_combine(const float* sst, const float* tproj, float* out, int N, int B, int D,
+                               const LaunchCtx& ctx) {
+    const long long total = (long long)N * B * 6 * D;
+    if (total <= 0) return cudaSuccess;
+    long long g = (total + 255) / 256;
+    if (g > ctx.num_sms * 8) g = ctx.num_sms * 8;
+    mod_combine_kernel<<<(int)g, 256, 0, ctx.stream>>>(sst, tproj, out, N, B, D);
     if (ctx.launches) ++*ctx.launches;
     return cudaGetLastError();
 }

@@ -101,14 +101,18 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
             for (int i = 0; i < 4; ++i) xu[i] = xp[i];
             float g[32];
             if (KIND == EPI_GATE_RESIDUAL) {
-                const float4* g0 = reinterpret_cast<const float4*>(e.gate0 + c);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 a = __ldg(g0 + i);
-                    g[4 * i] = a.x;
-                    g[4 * i + 1] = a.y;
-                    g[4 * i + 2] = a.z;
-                    g[4 * i + 3] = a.w;
+                for (int i = 0; i < 32; ++i) g[i] = 0.0f;
+                if (e.gate0) {
+                    const float4* g0 = reinterpret_cast<const float4*>(e.gate0 + c);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 a = __ldg(g0 + i);
+                        g[4 * i] = a.x;
+                        g[4 * i + 1] = a.y;
+                        g[4 * i + 2] = a.z;
+                        g[4 * i + 3] = a.w;
+                    }
                 }
                 if (e.gate1) {
                     const float4* g1 =

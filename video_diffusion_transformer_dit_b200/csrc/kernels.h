@@ -58,7 +58,12 @@ cudaError_t launch_attention(const void* q, long long ldq, const void* k, long l
                              long long ldv, void* o, long long ldo, int B, int heads, int Lq, int Lk,
                              const LaunchCtx& ctx);
 
-// LayerNorm (+ modulation or affine).
+// Per-sample modulation of every block: out[n][b][6][D] = sst[n] + tproj[b] (+1 on the scale rows).
+cudaError_t launch_mod_combine(const float* sst, const float* tproj, float* out, int N, int B, int D,
+                               const LaunchCtx& ctx);
+
+// LayerNorm (+ modulation or affine); mode 0 modulation from table + rows, 1 affine,
+// 2 precombined rows (scale1 = 1 + scale, shift1).
 cudaError_t launch_layernorm(const void* x, void* y, int rows, int D, float eps, int mode, const float* gamma,
                              const float* beta, const float* shift0, const float* shift1, const float* scale0,
                              const float* scale1, int mod_div, long long mod_ld, const LaunchCtx& ctx);

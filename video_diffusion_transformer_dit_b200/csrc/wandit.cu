@@ -97,6 +97,7 @@ struct wan_dit {
     std::vector<BlockW> blocks;
     void *w_pe, *w_t1, *w_t2, *w_tp, *w_x1, *w_x2, *w_kv, *w_po;
     float *b_pe, *b_t1, *b_t2, *b_tp, *b_x1, *b_x2, *b_kv, *k2_gain, *sst_out, *b_po;
+    float* sst_all;       // [N, 6, D] block tables, contiguous
     // workspace
     char* ws = nullptr;
     size_t ws_bytes = 0;
@@ -106,6 +107,7 @@ struct wan_dit {
     float* vel_stage;     // f32 [R * out_ch * 4]
     void *X, *x, *y, *qkv, *o, *qc, *u, *th, *ctx, *kv, *tsin, *tsilu;
     float *temb, *tproj, *th32;
+    float* modc;          // [N, max_batch, 6, D] per-sample modulation of every block
     int* d_err = nullptr;
     // options / state
     bool use_graph = true;
@@ -174,10 +176,10 @@ wan_status build_weights(wan_dit* h) {
     sz(D * P_in, 1); sz(D, 0);
     sz(D * c.freq_dim, 1); sz(D, 0); sz(D * D, 1); sz(D, 0); sz(6 * D * D, 1); sz(6 * D, 0);
     sz(D * c.text_dim, 1); sz(D, 0); sz(D * D, 1); sz(D, 0);
-    sz(N * 2 * D * D, 1); sz(N * 2 * D, 0); sz(N * D, 0);
+    sz(N * 2 * D * D, 1); sz(N * 2 * D, 0); sz(N * D, 0); sz(N * 6 * D, 0);
     for (int i = 0; i < N; ++i) {
         sz(3 * D * D, 1); sz(3 * D, 0); sz(D * D, 1); sz(D, 0); sz(D * D, 1); sz(D, 0); sz(D * D, 1); sz(D, 0);
-        sz(Fd * D, 1); sz(Fd, 0); sz(D * Fd, 1); sz(D, 0); sz(2 * D, 0); sz(D, 0); sz(D, 0); sz(D, 0); sz(6 * D, 0);
+        sz(Fd * D, 1); sz(Fd, 0); sz(D * Fd, 1); sz(D, 0); sz(2 * D, 0); sz(D, 0); sz(D, 0); sz(D, 0);
     }
     sz(2 * D, 0); sz(P_out * D, 1); sz(P_out, 0);
     h->arena_bytes = total;
@@ -216,6 +218,7 @@ wan_status build_weights(wan_dit* h) {
     h->w_kv = take(N * 2 * D * D, 1);
     h->b_kv = (float*)take(N * 2 * D, 0);
     h->k2_gain = (float*)take(N * D, 0);
+    h->sst_all = (float*)take(N * 6 * D, 0);
     h->blocks.resize(N);
     for (int i = 0; i < N; ++i) {
         BlockW& b = h->blocks[i];
@@ -230,7 +233,7 @@ wan_status build_weights(wan_dit* h) {
         b.q2_gain = (float*)take(D, 0);
         b.n2_g = (float*)take(D, 0);
         b.n2_b = (float*)take(D, 0);
-        b.sst = (float*)take(6 * D, 0);
+        b.sst = h->sst_all + (long long)i * 6 * D;
         auto bf = [](void* base, long long elems) { return (void*)((char*)base + elems * 2); };
         auto f4 = [](float* base, long long elems) { return (void*)(base + elems); };
         add_slot(h, p + "scale_shift_table", b.sst, 0, {1, 6, D});
@@ -288,6 +291,7 @@ wan_status build_workspace(wan_dit* h) {
         {&h->tsin, (size_t)(R * c.freq_dim * 2)},      {&h->tsilu, (size_t)(R * D * 2)},
         {(void**)&h->temb, (size_t)(R * D * 4)},       {(void**)&h->tproj, (size_t)(R * 6 * D * 4)},
         {(void**)&h->th32, (size_t)(R * D * 4)},
+        {(void**)&h->modc, (size_t)((long long)N * c.max_batch * 6 * D * 4)},
     };
     size_t total = 0;
     for (auto& it : items) total += align_up(it.bytes, 1024);
@@ -372,6 +376,7 @@ cudaError_t issue_forward(wan_dit* h, const Shape& s, const Plan& plan, const La
         TRYK(WAN_KC_EMBEDDING, wan::launch_gemv(h->w_t1, h->b_t1, h->t_stage, 1, h->th32, D, B, D, c.freq_dim, 2, 1, ctx));
         TRYK(WAN_KC_EMBEDDING, wan::launch_gemv(h->w_t2, h->b_t2, h->th32, D, h->temb, D, B, D, D, 0, 0, ctx));
         TRYK(WAN_KC_EMBEDDING, wan::launch_gemv(h->w_tp, h->b_tp, h->temb, D, h->tproj, D6, B, 6 * D, D, 1, 0, ctx));
+        TRYK(WAN_KC_EMBEDDING, wan::launch_mod_combine(h->sst_all, h->tproj, h->modc, N, B, D, ctx));
         mod_div = L;
     } else {
         TRYK(WAN_KC_EMBEDDING, wan::launch_sinusoid_bf16(h->t_stage, R, c.freq_dim, h->tsin, ctx));
@@ -394,16 +399,22 @@ cudaError_t issue_forward(wan_dit* h, const Shape& s, const Plan& plan, const La
     for (int i = 0; i < N; ++i) {
         const BlockW& w = h->blocks[i];
         // 1. self-attention: norm1 + modulation (shift row 0, scale row 1)
-        TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, w.sst, h->tproj, w.sst + D,
-                                  h->tproj + D, mod_div, D6, ctx));
+        // per-sample: precombined rows of modc (1 + scale folded in); per-token: table + projection rows
+        const float* mc = h->modc + (long long)i * B * 6 * D;
+        if (!s.per_token)
+            TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 2, nullptr, nullptr, nullptr, mc,
+                                                         nullptr, mc + D, mod_div, D6, ctx));
+        else
+            TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, w.sst, h->tproj,
+                                                         w.sst + D, h->tproj + D, mod_div, D6, ctx));
         TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, w.wqkv, D, R, 3 * D, D, epi(wan::EPI_BIAS, w.bqkv, h->qkv, 3LL * D), ctx));
         TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rmsnorm_rope(h->qkv, 3LL * D, R, D, c.eps, w.qk_gain, D, 2, D, &plan.rt, L, ctx));
         TRYK(WAN_KC_SELF_ATTENTION, wan::launch_attention(qkv, 3LL * D, qkv + 2LL * D, 3LL * D, qkv + 4LL * D, 3LL * D, h->o, D, B, c.heads, L,
                                   L, ctx));
         {
             EpiParams p = epi(wan::EPI_GATE_RESIDUAL, w.bo, h->x, D);
-            p.gate0 = w.sst + 2 * D;
-            p.gate1 = h->tproj + 2 * D;
+            p.gate0 = s.per_token ? w.sst + 2 * D : nullptr;
+            p.gate1 = s.per_token ? h->tproj + 2 * D : mc + 2 * D;
             p.mod_div = mod_div;
             p.mod_ld = D6;
             TRYK(WAN_KC_GEMM, wan::launch_gemm(h->o, D, w.wo, D, R, D, D, p, ctx));
@@ -417,13 +428,18 @@ cudaError_t issue_forward(wan_dit* h, const Shape& s, const Plan& plan, const La
         TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_attention(h->qc, D, kvb, ldkv, kvb + 2LL * D, ldkv, h->o, D, B, c.heads, L, Lc, ctx));
         TRYK(WAN_KC_GEMM, wan::launch_gemm(h->o, D, w.wo2, D, R, D, D, epi(wan::EPI_RESIDUAL, w.bo2, h->x, D), ctx));
         // 3. feed-forward: norm3 + modulation (shift row 3, scale row 4), GELU-tanh, gated residual (row 5)
-        TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, w.sst + 3 * D, h->tproj + 3 * D,
-                                  w.sst + 4 * D, h->tproj + 4 * D, mod_div, D6, ctx));
+        if (!s.per_token)
+            TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 2, nullptr, nullptr, nullptr, mc + 3 * D,
+                                                         nullptr, mc + 4 * D, mod_div, D6, ctx));
+        else
+            TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, w.sst + 3 * D,
+                                                         h->tproj + 3 * D, w.sst + 4 * D, h->tproj + 4 * D, mod_div, D6,
+                                                         ctx));
         TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, w.w1, D, R, Fd, D, epi(wan::EPI_BIAS_GELU, w.b1, h->u, Fd), ctx));
         {
             EpiParams p = epi(wan::EPI_GATE_RESIDUAL, w.b2, h->x, D);
-            p.gate0 = w.sst + 5 * D;
-            p.gate1 = h->tproj + 5 * D;
+            p.gate0 = s.per_token ? w.sst + 5 * D : nullptr;
+            p.gate1 = s.per_token ? h->tproj + 5 * D : mc + 5 * D;
             p.mod_div = mod_div;
             p.mod_ld = D6;
             TRYK(WAN_KC_GEMM, wan::launch_gemm(h->u, Fd, w.w2, Fd, R, D, Fd, p, ctx));
