@@ -5,14 +5,16 @@
 //
 // One CTA per (256 queries = two 128-row tiles, head, batch), 12 warps in
 // three warpgroups; the first gives registers to the two softmax groups
-// (56 / 224 / 224 per thread, 64512 in all = 384 threads x 168 at launch):
+// (88 / 208 / 208 per thread, 64512 in all = 384 threads x 168 at launch):
 //   warp 0      TMA producer: both Q tiles once, then K and V tiles of 128
 //               keys in two-slot rings (3-D tensor maps: rows past the
 //               sequence read as zero);
 //   warp 1      tensor-memory owner and MMA issuer.  Tensor memory holds
 //               S0 | S1 | O0 | O1 (4 x 128 fp32 columns).  Per key tile j it
 //               issues  PV0(j-1) S0(j) PV1(j-1) S1(j)  in that order, so the
-//               commit that publishes S_t(j) also covers PV_t(j-1);
+//               commit that publishes S_t(j) also covers PV_t(j-1); each P.V
+//               goes in two K = 64 halves, the first as soon as the softmax
+//               has stored the probabilities of keys 0..63;
 //   warps 2..3  idle;
 //   warps 4..7  softmax of tile 0, warps 8..11 softmax of tile 1 (one query
 //               row per thread, the two groups ping-pong with the tensor
@@ -53,8 +55,8 @@ constexpr int SMEM_BYTES = SBAR + 256 + 1024;
 constexpr int THREADS = 384;
 constexpr int REGS_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
 #ifndef WAN_ATTN_REGS_CONTROL
-#define WAN_ATTN_REGS_CONTROL 56
-#define WAN_ATTN_REGS_SOFTMAX 224
+#define WAN_ATTN_REGS_CONTROL 88
+#define WAN_ATTN_REGS_SOFTMAX 208
 #endif
 constexpr int REGS_CONTROL = WAN_ATTN_REGS_CONTROL;  // warpgroup 0: producer + MMA issuer
 constexpr int REGS_SOFTMAX = WAN_ATTN_REGS_SOFTMAX;  // warpgroups 1, 2
@@ -67,6 +69,10 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 #define WAN_ATTN_EX2_F32 1   // 1: one ex2.approx.f32 per exponential; 0: ex2.approx.f16x2 pairs (measured slower)
 #endif
 constexpr int EMU_PAIRS_OF_8 = WAN_ATTN_EMU_PAIRS;  // column pairs per 8 on the software exp2
+#ifndef WAN_ATTN_PV_SPLIT
+#define WAN_ATTN_PV_SPLIT 1
+#endif
+constexpr bool PV_SPLIT = WAN_ATTN_PV_SPLIT;  // P.V issued in two halves over the keys
 }  // namespace attn
 
 __global__ void __launch_bounds__(attn::THREADS, 1)
@@ -82,7 +88,8 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
     uint64_t* v_full = k_empty + KSTAGES;        // [VSTAGES]
     uint64_t* v_empty = v_full + VSTAGES;        // [VSTAGES]
     uint64_t* s_full = v_empty + VSTAGES;        // [2] per query tile
-    uint64_t* p_full = s_full + 2;               // [2]
+    uint64_t* p_half = s_full + 2;               // [2] P columns of keys 0..63 written
+    uint64_t* p_full = p_half + 2;               // [2]
     uint64_t* o_final = p_full + 2;              // [2]
     uint64_t* drain = o_final + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -106,6 +113,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(s_full + t, 1);
+            mbar_init(p_half + t, 4);
             mbar_init(p_full + t, 4);
             mbar_init(o_final + t, 1);
         }
@@ -162,59 +170,84 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- MMA issuer ----------------
-            constexpr uint32_t ID_QK = idesc_bf16(128, 128, false);
-            constexpr uint32_t ID_PV = idesc_bf16(128, 128, true);
-            const uint32_t sq = smem_u32(smem + SQ);
-            bool ok = mbar_wait(q_full, 0, abort_flag, p.wc);
-            bool issued = false;
-            // S_t(j) = Q_t K_j^T into TMEM columns [128 t, 128 t + 128)
-            auto issue_s = [&](int t, int j) -> bool {
-                const int ks = j % KSTAGES;
-                if (t == 0 && !mbar_wait(k_full + ks, (j / KSTAGES) & 1, abort_flag, p.wc)) return false;
-                tc_fence_after();
-                const uint32_t sk = smem_u32(smem + SK + ks * TILE_BYTES);
-                const uint32_t sqt = sq + t * TILE_BYTES;
+        // ---------------- MMA issuer ----------------
+        // The whole warp runs this loop (warp-uniform state); lane 0 waits on the
+        // barriers, one elected lane issues each group of MMAs and its commits.
+        // The issuing warp shares its SM sub-partition with two busy softmax
+        // warps, so every instruction between MMAs is kept out of the loop:
+        // descriptors are built once and moved by adding the offset (>> 4) to
+        // their start-address field.
+        constexpr uint32_t ID_QK = idesc_bf16(128, 128, false);
+        constexpr uint32_t ID_PV = idesc_bf16(128, 128, true);
+        const uint64_t dq = sdesc_kmajor_sw128(smem_u32(smem + SQ));
+        const uint64_t dk = sdesc_kmajor_sw128(smem_u32(smem + SK));
+        const uint64_t dv = sdesc_mnmajor_sw128(smem_u32(smem + SV), HALF_BYTES);
+        auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            int r = 1;
+            if (lane == 0) r = mbar_wait(bar, parity, abort_flag, p.wc) ? 1 : 0;
+            return __shfl_sync(0xffffffffu, r, 0) != 0;
+        };
+        bool ok = wait(q_full, 0);
+        bool issued = false;
+        // S_t(j) = Q_t K_j^T into TMEM columns [128 t, 128 t + 128)
+        auto issue_s = [&](int t, int j) -> bool {
+            const int ks = j % KSTAGES;
+            if (t == 0 && !wait(k_full + ks, (j / KSTAGES) & 1)) return false;
+            tc_fence_after();
+            const uint64_t a = dq + (uint64_t)((t * TILE_BYTES) >> 4);
+            const uint64_t b = dk + (uint64_t)((ks * TILE_BYTES) >> 4);
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-                    umma_bf16_ss(tmem + t * 128, sdesc_kmajor_sw128(sqt + off), sdesc_kmajor_sw128(sk + off), ID_QK,
-                                 kk != 0);
+                    const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+                    umma_bf16_ss(tmem + t * 128, a + off, b + off, ID_QK, kk != 0);
                 }
-                issued = true;
                 umma_commit(s_full + t);
                 if (t == 1) umma_commit(k_empty + ks);
-                return true;
-            };
-            // O_t += P_t(j) V_j, P_t read from the S_t columns (bf16 pairs)
-            auto issue_pv = [&](int t, int j) -> bool {
-                const int vs = j % VSTAGES;
-                if (!mbar_wait(p_full + t, j & 1, abort_flag, p.wc)) return false;
-                if (t == 0 && !mbar_wait(v_full + vs, (j / VSTAGES) & 1, abort_flag, p.wc)) return false;
-                tc_fence_after();
-                const uint32_t sv = smem_u32(smem + SV + vs * TILE_BYTES);
+            }
+            __syncwarp();
+            issued = true;
+            return true;
+        };
+        // O_t += P_t(j) V_j, P_t read from the S_t columns (bf16 pairs); with
+        // PV_SPLIT in two halves over the keys: keys 0..63 as soon as their
+        // probabilities are stored (p_half), keys 64..127 after the row (p_full)
+        auto issue_pv = [&](int t, int j, int k0, int k1, bool last) -> bool {
+            const int vs = j % VSTAGES;
+            if (!wait((last ? p_full : p_half) + t, j & 1)) return false;
+            if (t == 0 && k0 == 0 && !wait(v_full + vs, (j / VSTAGES) & 1)) return false;
+            tc_fence_after();
+            const uint64_t b = dv + (uint64_t)((vs * TILE_BYTES) >> 4);
+            const uint32_t acc0 = (j | k0) != 0;
+            if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    umma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                                 sdesc_mnmajor_sw128(sv + kk * 2048, HALF_BYTES), ID_PV, (j | kk) != 0);
+                for (int kk = k0; kk < k1; ++kk)
+                    umma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b + ((kk * 2048) >> 4), ID_PV,
+                                 kk == k0 ? acc0 : 1u);
+                if (last) {
+                    if (t == 1) umma_commit(v_empty + vs);
+                    if (j == nk - 1) umma_commit(o_final + t);
                 }
-                if (t == 1) umma_commit(v_empty + vs);
-                if (j == nk - 1) umma_commit(o_final + t);
-                return true;
-            };
-            if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
-            for (int j = 0; ok && j < nk; ++j) {
-                if (!issue_pv(0, j)) { ok = false; break; }
-                if (j + 1 < nk && !issue_s(0, j + 1)) { ok = false; break; }
-                if (!issue_pv(1, j)) { ok = false; break; }
-                if (j + 1 < nk && !issue_s(1, j + 1)) { ok = false; break; }
             }
-            if (!ok && issued) {  // let the tensor core finish before TMEM is freed
-                umma_commit(drain);
-                mbar_drain(drain, 0, 200000000ull);
-            }
+            __syncwarp();
+            return true;
+        };
+        auto issue_pv_all = [&](int t, int j) -> bool {
+            if (PV_SPLIT) return issue_pv(t, j, 0, 4, false) && issue_pv(t, j, 4, 8, true);
+            return issue_pv(t, j, 0, 8, true);
+        };
+        if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
+        for (int j = 0; ok && j < nk; ++j) {
+            if (!issue_pv_all(0, j)) { ok = false; break; }
+            if (j + 1 < nk && !issue_s(0, j + 1)) { ok = false; break; }
+            if (!issue_pv_all(1, j)) { ok = false; break; }
+            if (j + 1 < nk && !issue_s(1, j + 1)) { ok = false; break; }
         }
+        if (!ok && issued && elect_one()) {  // let the tensor core finish before TMEM is freed
+            umma_commit(drain);
+            mbar_drain(drain, 0, 200000000ull);
+        }
+        __syncwarp();
     }
     } else {
         regs_alloc<REGS_SOFTMAX>();
@@ -260,6 +293,20 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             const float m_new = fmaxf(m_run, m_tile);
             const bool rescale = m_new > m_run + RESCALE_THRESHOLD;
             const float m_use = rescale ? m_new : m_run;
+            // O_t is idle here (the commit of S_t(j) also covered P_t(j-1) V_{j-1}) and
+            // must be rescaled before the first half of P_t(j) V_j is issued
+            const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;  // 0 on the first tile
+            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(TO + c * 32, ov);
+                    tmem_ld_wait(ov);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                    tmem_st32(TO + c * 32, ov);
+                }
+            }
             // probabilities on packed fp32 pairs, EMU_PAIRS_OF_8 of every 8 pairs on the
             // software exp2 (FMA pipe); each 32-column chunk is packed to bf16 and
             // stored over its own S columns (P_t = first 64 columns of S_t) at once
@@ -289,23 +336,16 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     pc[i / 2] = pack_bf16(e0, e1);
                 }
                 tmem_st16(TS + c * 16, pc);
+                if (PV_SPLIT && c == 1) {  // keys 0..63 (and any O rescale) in tensor memory: first half of P.V may start
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(p_half + t);
+                }
             }
             float ps[4];
             f2unpack(ps2[0], ps[0], ps[1]);
             f2unpack(ps2[1], ps[2], ps[3]);
-            // O_t is idle here: the commit of S_t(j) also covered P_t(j-1) V_{j-1}
-            const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;  // 0 on the first tile
-            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t ov[32];
-                    tmem_ld32(TO + c * 32, ov);
-                    tmem_ld_wait(ov);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st32(TO + c * 32, ov);
-                }
-            }
             tmem_st_wait();
             if (rescale) {
                 l_run *= alpha;

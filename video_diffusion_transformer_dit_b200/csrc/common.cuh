@@ -53,11 +53,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                  : "memory");
 }
 
+#ifndef WAN_MBAR_TEST_WAIT
+#define WAN_MBAR_TEST_WAIT 1
+#endif
+// Non-blocking probe of a phase (test_wait): the first look of every wait.
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
+#if WAN_MBAR_TEST_WAIT
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+#else
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+#endif
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
@@ -276,6 +284,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
            | ((b_mn_major ? 1u : 0u) << 16)       // B major
            | ((static_cast<uint32_t>(N) >> 3) << 17)
            | ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+
+// True in exactly one lane of a fully converged warp (elect.sync over all 32 lanes).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.b32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 // Named barrier over `count` threads (a multiple of 32), id 1..15.
