@@ -62,17 +62,19 @@ constexpr int REGS_CONTROL = WAN_ATTN_REGS_CONTROL;  // warpgroup 0: producer + 
 constexpr int REGS_SOFTMAX = WAN_ATTN_REGS_SOFTMAX;  // warpgroups 1, 2
 static_assert(128 * REGS_CONTROL + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH, "register split");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+// Column pairs per 8 whose exp2 runs as the FMA-pipe cubic instead of on the
+// MUFU.  0 by default: scalar FP32 work in the softmax warps competes with the
+// MMA-issuing warp on the same sub-partitions (measured: a tight tcgen05.mma
+// issue loop drops to a third of the tensor rate next to FFMA-bound warps, and
+// is unaffected by MUFU-, integer- or packed-f32x2-bound ones), which costs
+// more than the MUFU time the emulation saves.
 #ifndef WAN_ATTN_EMU_PAIRS
-#define WAN_ATTN_EMU_PAIRS 2
+#define WAN_ATTN_EMU_PAIRS 0
 #endif
 #ifndef WAN_ATTN_EX2_F32
 #define WAN_ATTN_EX2_F32 1   // 1: one ex2.approx.f32 per exponential; 0: ex2.approx.f16x2 pairs (measured slower)
 #endif
 constexpr int EMU_PAIRS_OF_8 = WAN_ATTN_EMU_PAIRS;  // column pairs per 8 on the software exp2
-#ifndef WAN_ATTN_PV_SPLIT
-#define WAN_ATTN_PV_SPLIT 1
-#endif
-constexpr bool PV_SPLIT = WAN_ATTN_PV_SPLIT;  // P.V issued in two halves over the keys
 }  // namespace attn
 
 __global__ void __launch_bounds__(attn::THREADS, 1)
@@ -209,9 +211,9 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             issued = true;
             return true;
         };
-        // O_t += P_t(j) V_j, P_t read from the S_t columns (bf16 pairs); with
-        // PV_SPLIT in two halves over the keys: keys 0..63 as soon as their
-        // probabilities are stored (p_half), keys 64..127 after the row (p_full)
+        // O_t += P_t(j) V_j, P_t read from the S_t columns (bf16 pairs), in two
+        // halves over the keys: keys 0..63 as soon as their probabilities are
+        // stored (p_half), keys 64..127 after the whole row (p_full)
         auto issue_pv = [&](int t, int j, int k0, int k1, bool last) -> bool {
             const int vs = j % VSTAGES;
             if (!wait((last ? p_full : p_half) + t, j & 1)) return false;
@@ -233,8 +235,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             return true;
         };
         auto issue_pv_all = [&](int t, int j) -> bool {
-            if (PV_SPLIT) return issue_pv(t, j, 0, 4, false) && issue_pv(t, j, 4, 8, true);
-            return issue_pv(t, j, 0, 8, true);
+            return issue_pv(t, j, 0, 4, false) && issue_pv(t, j, 4, 8, true);
         };
         if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
         for (int j = 0; ok && j < nk; ++j) {
@@ -307,8 +308,8 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     tmem_st32(TO + c * 32, ov);
                 }
             }
-            // probabilities on packed fp32 pairs, EMU_PAIRS_OF_8 of every 8 pairs on the
-            // software exp2 (FMA pipe); each 32-column chunk is packed to bf16 and
+            // probabilities on packed fp32 pairs (EMU_PAIRS_OF_8 of every 8 pairs on the
+            // software exp2); each 32-column chunk is packed to bf16 and
             // stored over its own S columns (P_t = first 64 columns of S_t) at once
             uint64_t ps2[2] = {0ull, 0ull};
             const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     pc[i / 2] = pack_bf16(e0, e1);
                 }
                 tmem_st16(TS + c * 16, pc);
-                if (PV_SPLIT && c == 1) {  // keys 0..63 (and any O rescale) in tensor memory: first half of P.V may start
+                if (c == 1) {  // keys 0..63 (and any O rescale) in tensor memory: first half of P.V may start
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();

@@ -359,6 +359,11 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -397,6 +402,18 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
     const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
     const float k1 = 0.044715f;
     return 0.5f * x * (1.0f + tanh_approx(k0 * (x + k1 * x * x * x)));
+}
+// GELU (tanh form) of a packed fp32 pair: the polynomial on f32x2 operations,
+// tanh on the MUFU, so the scalar FP32 pipe stays free.
+__device__ __forceinline__ uint64_t gelu_tanh_f2(uint64_t x2) {
+    const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+    const float k1 = 0.044715f;
+    const uint64_t xx = mul2(x2, x2);
+    const uint64_t u = mul2(fma2(xx, f2pack(k0 * k1, k0 * k1), f2pack(k0, k0)), x2);  // k0 (x + k1 x^3)
+    float u0, u1;
+    f2unpack(u, u0, u1);
+    const uint64_t hx = mul2(x2, f2pack(0.5f, 0.5f));
+    return fma2(hx, f2pack(tanh_approx(u0), tanh_approx(u1)), hx);  // x/2 (1 + tanh u)
 }
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);

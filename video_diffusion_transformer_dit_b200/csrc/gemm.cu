@@ -52,9 +52,104 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmParams& p, int& 
     }
 }
 
+// Hot epilogues on packed fp32 pairs.  The accumulator columns arrive as 16
+// pairs; bias, GELU, gate and residual run as f32x2 operations, which keeps
+// the scalar FP32 pipe free for the MMA-issuing warp on the same SM
+// sub-partitions (scalar FFMA traffic there slows tcgen05.mma issue).
+template <int KIND>
+__device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, int c, const uint32_t (&r)[32]) {
+    uint64_t v2[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v2[i] = f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+    if (e.bias) {
+        const ulonglong2* b2 = reinterpret_cast<const ulonglong2*>(e.bias + c);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const ulonglong2 b = __ldg(b2 + i);
+            v2[2 * i] = add2(v2[2 * i], b.x);
+            v2[2 * i + 1] = add2(v2[2 * i + 1], b.y);
+        }
+    }
+    if (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU) {
+        if (KIND == EPI_BIAS_GELU) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v2[i] = gelu_tanh_f2(v2[i]);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                float a, b;
+                f2unpack(v2[4 * i + h], a, b);
+                w[h] = pack_bf16(a, b);
+            }
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    } else {  // EPI_GATE_RESIDUAL, EPI_RESIDUAL
+        // issue every load of the chunk before any store: x (4 x 16 B) and the gate rows
+        uint4* xp = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
+        uint4 xu[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xu[i] = xp[i];
+        uint64_t g2[16];
+        if (KIND == EPI_GATE_RESIDUAL) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) g2[i] = 0ull;  // +0.0f, +0.0f
+            if (e.gate1) {
+                const ulonglong2* g =
+                    reinterpret_cast<const ulonglong2*>(e.gate1 + (long long)(row / e.mod_div) * e.mod_ld + c);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const ulonglong2 a = __ldg(g + i);
+                    g2[2 * i] = a.x;
+                    g2[2 * i + 1] = a.y;
+                }
+            }
+            if (e.gate0) {
+                const ulonglong2* g = reinterpret_cast<const ulonglong2*>(e.gate0 + c);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const ulonglong2 a = __ldg(g + i);
+                    g2[2 * i] = add2(g2[2 * i], a.x);
+                    g2[2 * i + 1] = add2(g2[2 * i + 1], a.y);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t xw[4] = {xu[i].x, xu[i].y, xu[i].z, xu[i].w};
+            uint32_t ow[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 xf = unpack_bf16(xw[h]);
+                const uint64_t x2 = f2pack(xf.x, xf.y);
+                uint64_t o2;
+                if (KIND == EPI_GATE_RESIDUAL) {
+                    o2 = fma2(v2[4 * i + h], g2[4 * i + h], x2);
+                } else {  // the branch output is rounded to bf16 before the residual add
+                    float a, b;
+                    f2unpack(v2[4 * i + h], a, b);
+                    const float2 ab = unpack_bf16(pack_bf16(a, b));
+                    o2 = add2(x2, f2pack(ab.x, ab.y));
+                }
+                float a, b;
+                f2unpack(o2, a, b);
+                ow[h] = pack_bf16(a, b);
+            }
+            xp[i] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        }
+    }
+}
+
 // Epilogue of 32 consecutive columns [c, c + 32) of one row (KIND fixed at compile time).
 template <int KIND>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int c, const uint32_t (&r)[32]) {
+    if (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU || KIND == EPI_GATE_RESIDUAL || KIND == EPI_RESIDUAL) {
+        epilogue_chunk_f2<KIND>(e, row, c, r);
+        return;
+    }
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
