@@ -75,6 +75,13 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 #define WAN_ATTN_EX2_F32 1   // 1: one ex2.approx.f32 per exponential; 0: ex2.approx.f16x2 pairs (measured slower)
 #endif
 constexpr int EMU_PAIRS_OF_8 = WAN_ATTN_EMU_PAIRS;  // column pairs per 8 on the software exp2
+#ifndef WAN_ATTN_PV_PARTS
+#define WAN_ATTN_PV_PARTS 2
+#endif
+// P.V issued in 2 or 4 parts over the 128 keys of a tile (measured at the 480p
+// shape: 2 parts ~1210 TFLOP/s, 4 parts ~1035, one part ~1060 with this issuer)
+constexpr int PV_PARTS = WAN_ATTN_PV_PARTS;
+static_assert(PV_PARTS == 2 || PV_PARTS == 4, "PV_PARTS");
 }  // namespace attn
 
 __global__ void __launch_bounds__(attn::THREADS, 1)
@@ -90,8 +97,8 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
     uint64_t* v_full = k_empty + KSTAGES;        // [VSTAGES]
     uint64_t* v_empty = v_full + VSTAGES;        // [VSTAGES]
     uint64_t* s_full = v_empty + VSTAGES;        // [2] per query tile
-    uint64_t* p_half = s_full + 2;               // [2] P columns of keys 0..63 written
-    uint64_t* p_full = p_half + 2;               // [2]
+    uint64_t* p_part = s_full + 2;               // [2][PV_PARTS - 1] P columns of the first parts written
+    uint64_t* p_full = p_part + 2 * (PV_PARTS - 1);  // [2]
     uint64_t* o_final = p_full + 2;              // [2]
     uint64_t* drain = o_final + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -115,7 +122,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(s_full + t, 1);
-            mbar_init(p_half + t, 4);
+            for (int q = 0; q < PV_PARTS - 1; ++q) mbar_init(p_part + t * (PV_PARTS - 1) + q, 4);
             mbar_init(p_full + t, 4);
             mbar_init(o_final + t, 1);
         }
@@ -211,12 +218,13 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             issued = true;
             return true;
         };
-        // O_t += P_t(j) V_j, P_t read from the S_t columns (bf16 pairs), in two
-        // halves over the keys: keys 0..63 as soon as their probabilities are
-        // stored (p_half), keys 64..127 after the whole row (p_full)
-        auto issue_pv = [&](int t, int j, int k0, int k1, bool last) -> bool {
+        // O_t += P_t(j) V_j, P_t read from the S_t columns (bf16 pairs), in
+        // PV_PARTS parts over the keys, each issued as soon as the softmax has
+        // stored its probabilities (p_part), the last after the whole row (p_full)
+        auto issue_pv = [&](int t, int j, int k0, int k1, uint64_t* bar) -> bool {
             const int vs = j % VSTAGES;
-            if (!wait((last ? p_full : p_half) + t, j & 1)) return false;
+            const bool last = k1 == 8;
+            if (!wait(bar, j & 1)) return false;
             if (t == 0 && k0 == 0 && !wait(v_full + vs, (j / VSTAGES) & 1)) return false;
             tc_fence_after();
             const uint64_t b = dv + (uint64_t)((vs * TILE_BYTES) >> 4);
@@ -235,7 +243,12 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             return true;
         };
         auto issue_pv_all = [&](int t, int j) -> bool {
-            return issue_pv(t, j, 0, 4, false) && issue_pv(t, j, 4, 8, true);
+#pragma unroll
+            for (int q = 0; q < PV_PARTS; ++q) {
+                uint64_t* bar = q == PV_PARTS - 1 ? p_full + t : p_part + t * (PV_PARTS - 1) + q;
+                if (!issue_pv(t, j, q * 8 / PV_PARTS, (q + 1) * 8 / PV_PARTS, bar)) return false;
+            }
+            return true;
         };
         if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
         for (int j = 0; ok && j < nk; ++j) {
@@ -337,11 +350,11 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     pc[i / 2] = pack_bf16(e0, e1);
                 }
                 tmem_st16(TS + c * 16, pc);
-                if (c == 1) {  // keys 0..63 (and any O rescale) in tensor memory: first half of P.V may start
+                if (c < 3 && (c + 1) % (4 / PV_PARTS) == 0) {  // a part of P (and any O rescale) stored: its P.V may start
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(p_half + t);
+                    if (lane == 0) mbar_arrive(p_part + t * (PV_PARTS - 1) + (c + 1) / (4 / PV_PARTS) - 1);
                 }
             }
             float ps[4];

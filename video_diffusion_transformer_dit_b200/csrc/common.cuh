@@ -370,27 +370,32 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
     return d;
 }
 
-// 2^x for a pair of x <= 8 on the FMA and integer pipes instead of the MUFU:
-// x = n + f with n the nearest integer (magic-number rounding) and |f| <= 1/2,
-// p(f) ~ 2^f from a cubic fitted by weighted least squares on Chebyshev nodes
-// (coefficients from gen_exp2_poly.py, relative error < 8e-5), then n added to
-// the exponent field.  x is clamped at -125 so the exponent never underflows
-// (2^-125 ~ 2e-38 stands in for 0).
+// 2^x for a pair of x <= 8 without the MUFU and without scalar FP32 or
+// integer-multiply work (which would compete with tcgen05.mma issue on the
+// same SM sub-partition): x = n + f with n the nearest integer (magic-number
+// rounding on packed f32x2 adds) and |f| <= 1/2; p(f) ~ 2^f from a cubic
+// fitted by weighted least squares on Chebyshev nodes (coefficients from
+// gen_exp2_poly.py, relative error < 8e-5), evaluated with packed FMAs; 2^n
+// built by inserting the biased exponent n + 127 (the low byte of the rounded
+// sum) into an empty word with bfi, applied with one packed multiply.  x is
+// clamped at -125 so the exponent never underflows (2^-125 ~ 2e-38 stands
+// in for 0).
 __device__ __forceinline__ void ex2_poly2(uint64_t x2, float& e0, float& e1) {
     float x0, x1;
     f2unpack(x2, x0, x1);
     const uint64_t xc = f2pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-    const uint64_t magic = f2pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-    const uint64_t t2 = add2(xc, magic);
+    const uint64_t magic = f2pack(12583039.0f, 12583039.0f);  // 1.5 * 2^23 + 127
+    const uint64_t t2 = add2(xc, magic);                        // low byte of the bits: n + 127
     const uint64_t fr = sub2(xc, sub2(t2, magic));
     uint64_t p2 = fma2(f2pack(5.508868396e-02f, 5.508868396e-02f), fr, f2pack(2.426040471e-01f, 2.426040471e-01f));
     p2 = fma2(p2, fr, f2pack(6.932762265e-01f, 6.932762265e-01f));
     p2 = fma2(p2, fr, f2pack(9.999289513e-01f, 9.999289513e-01f));
-    float p0, p1, t0, t1;
-    f2unpack(p2, p0, p1);
+    float t0, t1;
     f2unpack(t2, t0, t1);
-    e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+    uint32_t s0, s1;
+    asm("bfi.b32 %0, %1, 0, 23, 8;" : "=r"(s0) : "r"(__float_as_uint(t0)));
+    asm("bfi.b32 %0, %1, 0, 23, 8;" : "=r"(s1) : "r"(__float_as_uint(t1)));
+    f2unpack(mul2(p2, f2pack(__uint_as_float(s0), __uint_as_float(s1))), e0, e1);
 }
 
 __device__ __forceinline__ float tanh_approx(float x) {

@@ -203,6 +203,83 @@ __global__ void __launch_bounds__(256) rmsnorm_rope_kernel(__nv_bfloat16* buf, l
     }
 }
 
+// q and k of one token in one warp (the self-attention case): both rows are
+// loaded before either reduction, and each cos/sin pair is fetched once for
+// the two rotations.  q = buf[row, 0:D), k = buf[row, seg_stride:seg_stride+D).
+__device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
+    const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y; v[4] = c.x; v[5] = c.y; v[6] = d.x; v[7] = d.y;
+}
+
+template <int NCH>
+__global__ void __launch_bounds__(256) rmsnorm_rope_qk_kernel(__nv_bfloat16* buf, long long ld, int rows, float eps,
+                                                              const float* gains, long long gain_stride,
+                                                              long long seg_stride, RopeTables rt, int rope_L) {
+    constexpr int D = NCH * 256;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= rows) return;
+    __nv_bfloat16* xq = buf + (long long)row * ld;
+    __nv_bfloat16* xk = xq + seg_stride;
+    uint4 uq[NCH], uk[NCH];
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) {
+        uq[t] = *reinterpret_cast<const uint4*>(xq + (t * 32 + lane) * 8);
+        uk[t] = *reinterpret_cast<const uint4*>(xk + (t * 32 + lane) * 8);
+    }
+    const int l = row % rope_L;
+    const int hw = rt.Hp * rt.Wp;
+    const int f = l / hw;
+    const int rem = l - f * hw;
+    const int ii = rem / rt.Wp;
+    const int jj = rem - ii * rt.Wp;
+    float sq = 0.f, sk = 0.f;
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) {
+        float a[8], b[8];
+        unpack8(uq[t], a);
+        unpack8(uk[t], b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            sq += a[i] * a[i];
+            sk += b[i] * b[i];
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        sk += __shfl_xor_sync(0xffffffffu, sk, o);
+    }
+    const float rq = rsqrtf(sq * (1.0f / D) + eps);
+    const float rk = rsqrtf(sk * (1.0f / D) + eps);
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) {
+        const int c = (t * 32 + lane) * 8;
+        float a[8], b[8], gq[8], gk[8];
+        unpack8(uq[t], a);
+        unpack8(uk[t], b);
+        load8f(gains + c, gq);
+        load8f(gains + gain_stride + c, gk);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            a[i] *= rq * gq[i];
+            b[i] *= rk * gk[i];
+        }
+        const int p0 = (c & 127) >> 1;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 cs = rope_cs(rt, p0 + k, f, ii, jj);
+            const float a0 = a[2 * k], a1 = a[2 * k + 1], b0 = b[2 * k], b1 = b[2 * k + 1];
+            a[2 * k] = a0 * cs.x - a1 * cs.y;
+            a[2 * k + 1] = a0 * cs.y + a1 * cs.x;
+            b[2 * k] = b0 * cs.x - b1 * cs.y;
+            b[2 * k + 1] = b0 * cs.y + b1 * cs.x;
+        }
+        store8(xq + c, a);
+        store8(xk + c, b);
+    }
+}
+
 cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float eps, const float* gains,
                                 long long gain_stride, int nseg, long long seg_stride, const RopeTables* rope,
                                 int rope_L, const LaunchCtx& ctx) {
@@ -217,8 +294,23 @@ cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float 
     } else {
         rope_L = 1;
     }
-    dim3 grid((rows + 7) / 8, nseg);
     auto Bp = reinterpret_cast<__nv_bfloat16*>(buf);
+    if (use_rope && nseg == 2) {
+#define WAN_RMS_QK_CASE(n)                                                                                     \
+    case n:                                                                                                    \
+        rmsnorm_rope_qk_kernel<n><<<(rows + 7) / 8, 256, 0, ctx.stream>>>(Bp, ld, rows, eps, gains, gain_stride, \
+                                                                           seg_stride, rt, rope_L);            \
+        break;
+        switch (D / 256) {
+            WAN_RMS_QK_CASE(1) WAN_RMS_QK_CASE(2) WAN_RMS_QK_CASE(3) WAN_RMS_QK_CASE(4) WAN_RMS_QK_CASE(6)
+            WAN_RMS_QK_CASE(8) WAN_RMS_QK_CASE(12) WAN_RMS_QK_CASE(16) WAN_RMS_QK_CASE(20) WAN_RMS_QK_CASE(24)
+            default: return cudaErrorInvalidValue;
+        }
+#undef WAN_RMS_QK_CASE
+        if (ctx.launches) ++*ctx.launches;
+        return cudaGetLastError();
+    }
+    dim3 grid((rows + 7) / 8, nseg);
 #define WAN_RMS_CASE(n)                                                                                           \
     case n:                                                                                                       \
         rmsnorm_rope_kernel<n><<<grid, 256, 0, ctx.stream>>>(Bp, ld, rows, eps, gains, gain_stride, seg_stride, rt, \

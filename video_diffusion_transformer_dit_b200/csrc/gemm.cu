@@ -146,10 +146,9 @@ __device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, i
 // Epilogue of 32 consecutive columns [c, c + 32) of one row (KIND fixed at compile time).
 template <int KIND>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int c, const uint32_t (&r)[32]) {
-    if (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU || KIND == EPI_GATE_RESIDUAL || KIND == EPI_RESIDUAL) {
+    if constexpr (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU || KIND == EPI_GATE_RESIDUAL || KIND == EPI_RESIDUAL) {
         epilogue_chunk_f2<KIND>(e, row, c, r);
-        return;
-    }
+    } else {
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
@@ -271,6 +270,7 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
         }
         default:
             break;
+    }
     }
 }
 
