@@ -22,6 +22,10 @@ __device__ __forceinline__ void load8f(const float* p, float (&v)[8]) {
     float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
+__device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
+    const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y; v[4] = c.x; v[5] = c.y; v[6] = d.x; v[7] = d.y;
+}
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -32,59 +36,65 @@ __device__ __forceinline__ float warp_sum(float x) {
 // mode 0: y = LN(x) * (1 + scale0 + scale1[m]) + shift0 + shift1[m]
 // mode 1: y = LN(x) * gamma + beta
 // mode 2: y = LN(x) * scale1[m] + shift1[m]   (modulation precombined, 1 + scale included)
-template <int NCH>
+template <int NCH, int MODE>
 __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y,
-                                                        int rows, float eps, int mode, const float* gamma,
-                                                        const float* beta, const float* shift0, const float* shift1,
-                                                        const float* scale0, const float* scale1, int mod_div,
-                                                        long long mod_ld) {
+                                                        int rows, float eps, const float* gamma, const float* beta,
+                                                        const float* shift0, const float* shift1, const float* scale0,
+                                                        const float* scale1, int mod_div, long long mod_ld) {
     constexpr int D = NCH * 256;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * 8 + warp;
     if (row >= rows) return;
     const __nv_bfloat16* xr = x + (long long)row * D;
-    float v[NCH][8];
+    uint4 u[NCH];  // the row stays packed (bf16) in registers between the passes
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) u[t] = *reinterpret_cast<const uint4*>(xr + (t * 32 + lane) * 8);
     float s = 0.f;
 #pragma unroll
     for (int t = 0; t < NCH; ++t) {
-        load8(xr + (t * 32 + lane) * 8, v[t]);
+        float v[8];
+        unpack8(u[t], v);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) s += v[t][i];
+        for (int i = 0; i < 8; ++i) s += v[i];
     }
     const float mean = warp_sum(s) * (1.0f / D);
     float ss = 0.f;
 #pragma unroll
-    for (int t = 0; t < NCH; ++t)
+    for (int t = 0; t < NCH; ++t) {
+        float v[8];
+        unpack8(u[t], v);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float d = v[t][i] - mean;
+            const float d = v[i] - mean;
             ss += d * d;
         }
+    }
     const float rstd = rsqrtf(warp_sum(ss) * (1.0f / D) + eps);
     const long long m = (long long)(row / mod_div) * mod_ld;
     __nv_bfloat16* yr = y + (long long)row * D;
 #pragma unroll
     for (int t = 0; t < NCH; ++t) {
         const int c = (t * 32 + lane) * 8;
-        float a[8], bb[8], o[8];
-        if (mode == 2) {
+        float v[8], a[8], bb[8], o[8];
+        unpack8(u[t], v);
+        if (MODE == 2) {
             load8f(scale1 + m + c, a);
             load8f(shift1 + m + c, bb);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = (v[t][i] - mean) * rstd * a[i] + bb[i];
-        } else if (mode == 0) {
+            for (int i = 0; i < 8; ++i) o[i] = (v[i] - mean) * rstd * a[i] + bb[i];
+        } else if (MODE == 0) {
             float s1[8], h1[8];
             load8f(scale0 + c, a);
             load8f(shift0 + c, bb);
             load8f(scale1 + m + c, s1);
             load8f(shift1 + m + c, h1);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = (v[t][i] - mean) * rstd * (1.0f + a[i] + s1[i]) + (bb[i] + h1[i]);
+            for (int i = 0; i < 8; ++i) o[i] = (v[i] - mean) * rstd * (1.0f + a[i] + s1[i]) + (bb[i] + h1[i]);
         } else {
             load8f(gamma + c, a);
             load8f(beta + c, bb);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = (v[t][i] - mean) * rstd * a[i] + bb[i];
+            for (int i = 0; i < 8; ++i) o[i] = (v[i] - mean) * rstd * a[i] + bb[i];
         }
         store8(yr + c, o);
     }
@@ -101,8 +111,15 @@ cudaError_t launch_layernorm(const void* x, void* y, int rows, int D, float eps,
     auto Y = reinterpret_cast<__nv_bfloat16*>(y);
 #define WAN_LN_CASE(n)                                                                                             \
     case n:                                                                                                        \
-        layernorm_kernel<n><<<grid, 256, 0, ctx.stream>>>(X, Y, rows, eps, mode, gamma, beta, shift0, shift1, scale0, \
-                                                          scale1, mod_div, mod_ld);                                \
+        if (mode == 2)                                                                                             \
+            layernorm_kernel<n, 2><<<grid, 256, 0, ctx.stream>>>(X, Y, rows, eps, gamma, beta, shift0, shift1,      \
+                                                                 scale0, scale1, mod_div, mod_ld);                 \
+        else if (mode == 0)                                                                                        \
+            layernorm_kernel<n, 0><<<grid, 256, 0, ctx.stream>>>(X, Y, rows, eps, gamma, beta, shift0, shift1,      \
+                                                                 scale0, scale1, mod_div, mod_ld);                 \
+        else                                                                                                       \
+            layernorm_kernel<n, 1><<<grid, 256, 0, ctx.stream>>>(X, Y, rows, eps, gamma, beta, shift0, shift1,      \
+                                                                 scale0, scale1, mod_div, mod_ld);                 \
         break;
     switch (D / 256) {
         WAN_LN_CASE(1) WAN_LN_CASE(2) WAN_LN_CASE(3) WAN_LN_CASE(4) WAN_LN_CASE(6) WAN_LN_CASE(8) WAN_LN_CASE(12)
@@ -206,10 +223,6 @@ __global__ void __launch_bounds__(256) rmsnorm_rope_kernel(__nv_bfloat16* buf, l
 // q and k of one token in one warp (the self-attention case): both rows are
 // loaded before either reduction, and each cos/sin pair is fetched once for
 // the two rotations.  q = buf[row, 0:D), k = buf[row, seg_stride:seg_stride+D).
-__device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
-    const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y; v[4] = c.x; v[5] = c.y; v[6] = d.x; v[7] = d.y;
-}
 
 template <int NCH>
 __global__ void __launch_bounds__(256) rmsnorm_rope_qk_kernel(__nv_bfloat16* buf, long long ld, int rows, float eps,
@@ -295,7 +308,7 @@ cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float 
         rope_L = 1;
     }
     auto Bp = reinterpret_cast<__nv_bfloat16*>(buf);
-    if (use_rope && nseg == 2) {
+    if (use_rope && nseg == 2 && D <= 3072) {  // wider rows: two rows per warp would not fit in registers
 #define WAN_RMS_QK_CASE(n)                                                                                     \
     case n:                                                                                                    \
         rmsnorm_rope_qk_kernel<n><<<(rows + 7) / 8, 256, 0, ctx.stream>>>(Bp, ld, rows, eps, gains, gain_stride, \
@@ -303,7 +316,7 @@ cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float 
         break;
         switch (D / 256) {
             WAN_RMS_QK_CASE(1) WAN_RMS_QK_CASE(2) WAN_RMS_QK_CASE(3) WAN_RMS_QK_CASE(4) WAN_RMS_QK_CASE(6)
-            WAN_RMS_QK_CASE(8) WAN_RMS_QK_CASE(12) WAN_RMS_QK_CASE(16) WAN_RMS_QK_CASE(20) WAN_RMS_QK_CASE(24)
+            WAN_RMS_QK_CASE(8) WAN_RMS_QK_CASE(12)
             default: return cudaErrorInvalidValue;
         }
 #undef WAN_RMS_QK_CASE
