@@ -72,9 +72,7 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 #define WAN_ATTN_EMU_PAIRS 0
 #endif
 #ifndef WAN_ATTN_EX2_F32
-// 1: one ex2.approx.f32 per exponential; 0: ex2.approx.f16x2 pairs (measured
-// slower, as is ex2.approx.ftz.bf16x2: ~745 against ~1200 TFLOP/s at the 480p shape)
-#define WAN_ATTN_EX2_F32 1
+#define WAN_ATTN_EX2_F32 1   // 1: one ex2.approx.f32 per exponential; 0: ex2.approx.f16x2 pairs (measured slower)
 #endif
 constexpr int EMU_PAIRS_OF_8 = WAN_ATTN_EMU_PAIRS;  // column pairs per 8 on the software exp2
 #ifndef WAN_ATTN_PV_PARTS
