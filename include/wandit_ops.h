@@ -47,8 +47,10 @@ typedef struct {
     void* out;            /* output (bf16 or f32 per epilogue); read too for the
                              residual epilogues                                  */
     int64_t ldo;          /* row stride of out in elements                        */
-    const float* gate0;   /* [N] f32 (gate epilogue)                              */
-    const float* gate1;   /* f32 rows of the per-sample / per-token modulation    */
+    const float* gate0;   /* [N] f32 (gate epilogue), or NULL (read as 0)         */
+    const float* gate1;   /* f32 rows of the per-sample / per-token modulation, or
+                             NULL (read as 0); the gate epilogue needs at least
+                             one of gate0, gate1 (else WAN_EINVAL)               */
     int mod_div;          /* modulation row = r / mod_div                         */
     int64_t mod_ld;       /* row stride of gate1 in elements                      */
     int up_C, up_F, up_Hz, up_Wz; /* unpatchify geometry, patch (1,2,2)           */

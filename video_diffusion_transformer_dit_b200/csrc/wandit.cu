@@ -867,7 +867,7 @@ wan_status wan_op_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, i
                        const wan_epilogue* ep, void* stream) {
     if (!A || !W || !ep || !ep->out) return WAN_EINVAL;
     if (epilogue < WAN_EPI_BIAS || epilogue > WAN_EPI_UNPATCHIFY) return WAN_EINVAL;
-    if (epilogue == WAN_EPI_GATE_RESIDUAL && !ep->gate0) return WAN_EINVAL;
+    if (epilogue == WAN_EPI_GATE_RESIDUAL && !ep->gate0 && !ep->gate1) return WAN_EINVAL;
     if (M < 0) return WAN_ESHAPE;
     EpiParams p{};
     p.kind = epilogue;
