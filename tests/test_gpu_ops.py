@@ -111,6 +111,28 @@ def test_gemm_gate_residual(per_token):
     assert rel_l2(xd, ref) < TOL
 
 
+def test_gemm_gate_residual_single_gate_vector():
+    # the per-sample form the forward uses: one precombined gate row per sample (gate0 absent),
+    # and the table-only form (gate1 absent)
+    M, N, K, L = 400, 256, 256, 200
+    A, W, bias = _gemm_inputs(M, N, K, seed=6)
+    g = torch.Generator().manual_seed(7)
+    x = torch.randn(M, N, generator=g).to(torch.bfloat16)
+    rows = torch.randn(2, 6, N, generator=g) * 0.1
+    lin = O.linear(A.to(DT), W.to(DT), bias.to(DT))
+    xd = x.cuda()
+    B().op_gemm(A.cuda(), W.cuda(), "gate_residual", xd, bias=bias.cuda(), gate1=rows[:, 2].contiguous().cuda(),
+                mod_div=L, mod_ld=N)
+    B().op_sync()
+    assert rel_l2(xd, x.to(DT) + lin * rows[:, 2].to(DT).repeat_interleave(L, 0)) < TOL
+    xd = x.cuda()
+    B().op_gemm(A.cuda(), W.cuda(), "gate_residual", xd, bias=bias.cuda(), gate0=rows[0, 5].contiguous().cuda())
+    B().op_sync()
+    assert rel_l2(xd, x.to(DT) + lin * rows[0, 5].to(DT)) < TOL
+    with pytest.raises(B().WanError):
+        B().op_gemm(A.cuda(), W.cuda(), "gate_residual", x.cuda(), bias=bias.cuda())
+
+
 def test_gemm_residual():
     M, N, K = 260, 384, 128
     A, W, bias = _gemm_inputs(M, N, K, seed=4)
