@@ -160,11 +160,22 @@ def whole_job_tokens_per_s(world, batch, tokens, ms_per_step):
     return world * batch * tokens / (ms_per_step * 1e-3)
 
 
+def arm_config(workload, world):
+    """The `config` object both arms print for a workload."""
+    from video_diffusion_transformer_dit_b200 import configs
+    w = configs.workload(workload)
+    cfg = w["cfg"]
+    B, Cc, F, Hz, Wz = w["latent"]
+    return {"workload": workload, "model": "Wan2.1-T2V-1.3B shape" if "1.3b" in workload else cfg,
+            "global_batch": world * B, "seq_len": F * (Hz // 2) * (Wz // 2), "text_len": w["text_len"],
+            "blocks": cfg["num_blocks"], "timesteps": w["timesteps"], "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (2.8 GB weights + GBs of activations per step); no flush"}
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
-    from oracle import wan_oracle as O  # noqa: F401  (token law only used via configs)
     from video_diffusion_transformer_dit_b200 import build, configs, synth
     from video_diffusion_transformer_dit_b200.binding import WAN_OPT_KERNEL_TIMING, WanDiT
 
@@ -269,10 +280,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic latents/contexts, random-init bf16 weights of the named shapes",
-        "config": {"workload": args.workload, "model": "Wan2.1-T2V-1.3B shape" if "1.3b" in args.workload else cfg,
-                   "global_batch": world * B, "seq_len": L, "text_len": Lc, "blocks": cfg["num_blocks"],
-                   "timesteps": w["timesteps"], "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (2.8 GB weights + GBs of activations per step); no flush"},
+        "config": arm_config(args.workload, world),
         "tflops_per_step": flops / 1e12,
         "achieved_tflops": flops / (ms * 1e-3) / 1e12,
         "tc_peak_frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
@@ -416,7 +424,7 @@ def main():
             "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload},
+            "config": arm_config(args.workload, world),
             "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }))
@@ -426,7 +434,7 @@ def main():
     import torch.distributed as dist
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
         res = run_ours(args, rank, world, local_rank)
         if rank == 0:
