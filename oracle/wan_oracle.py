@@ -44,12 +44,25 @@ R11 token order (f, i, j) row-major, j fastest.
 R12 patch feature order (c, kt, kh, kw), c slowest (Conv3d weight flatten).
 R13 proj_out feature order (kt, kh, kw, c), c fastest (unpatchify reshape).
 R14 per-token timestep: t of shape [B, L]; every modulation row per token.
+R19 I2V image embedder: the CLIP tokens [B, Li, 1280] pass an MLP to the model
+    width, taken in the text embedder's form L2(GELU_tanh(L1(c))) with L1
+    1280 -> D and L2 D -> D.
+R20 I2V image cross-attention: the image tokens (placed before the text tokens
+    in the model forward) are split off again in every block and attended
+    separately: own key/value projections, keys RMSNorm'd across heads like the
+    text keys, the queries of the text cross-attention; the two attention
+    outputs are summed before the shared output projection.
+R21 MoE expert switch: with t decreasing over sampling, steps with
+    t >= boundary * num_train_timesteps use the high-noise expert and the rest
+    the low-noise expert; both forwards of a CFG step use the same expert.
 
 Parity unpinned (conventions the pages do not fix, so no pin can tell a
 right reading from a wrong one; the oracle and the CUDA path simply agree):
 the choice of cos-before-sin and the 1e4 base of the sinusoid (R2), the
 activation inside the time MLP (R3), the interleaved-pair RoPE layout and its
-44/42/42 split (R7), and the init/gain conventions of the synthetic weights.
+44/42/42 split (R7), the form of the image MLP (R19) and the projections and
+norm of the image branch (R20), and the init/gain conventions of the synthetic
+weights.
 Everything else is pinned by ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
@@ -238,6 +251,28 @@ def text_embedding(context: torch.Tensor, W: Dict[str, torch.Tensor]) -> torch.T
     return linear(h, W[p + "linear_2.weight"], W[p + "linear_2.bias"])
 
 
+def image_embedding(image: torch.Tensor, W: Dict[str, torch.Tensor]) -> torch.Tensor:
+    """I2V ``condition_embedder`` image path: CLIP tokens [B, Li, 1280] -> [B, Li, D]
+    ([WAN21-GUIDE] §4 "T5与CLIP": 257 CLIP tokens of width 1280 projected to the
+    model width by an MLP; [ANIMATE-DIFF] "配置参数全解": image_dim 1280 for the
+    CLIP features; [PSWP-WAN] "WanTransformer3DModel": the image tokens come out
+    of the condition embedder next to the text tokens).  Reading R19."""
+    p = "condition_embedder.image_embedder."
+    h = gelu_tanh(linear(image.to(DT), W[p + "linear_1.weight"], W[p + "linear_1.bias"]))
+    return linear(h, W[p + "linear_2.weight"], W[p + "linear_2.bias"])
+
+
+def i2v_input(noisy: torch.Tensor, cond: torch.Tensor, mask: torch.Tensor) -> torch.Tensor:
+    """DiT input of the I2V route: noisy latent (z channels), first-frame
+    condition latent (z channels) and known-frame mask (4 channels) joined on the
+    channel axis, not the time axis: 2 z + 4 channels, 36 for z = 16
+    ([WAN21-GUIDE] §4 table "I2V分量"; [ANIMATE-DIFF] "配置参数全解":
+    in_channels 36 = 2 * latent_channels + 4)."""
+    if not (noisy.shape[2:] == cond.shape[2:] == mask.shape[2:]) or mask.shape[1] != 4:
+        raise ValueError("noisy, cond, mask must share (B, F, H, W); mask has 4 channels")
+    return torch.cat([noisy, cond, mask], dim=1)
+
+
 # --------------------------------------------------------------------------
 # 3-axis rotary position embedding
 # --------------------------------------------------------------------------
@@ -326,14 +361,25 @@ def self_attention(y, Wb, angles, cfg, rows=None):
     return linear(o, Wb["attn1.to_out.0.weight"], Wb["attn1.to_out.0.bias"])
 
 
-def cross_attention(yc, ctx, Wb, cfg):
+def cross_attention(yc, ctx, Wb, cfg, img=None):
     """``attn2``: queries from the video tokens, keys/values from the projected
-    text context ([WAN21-GUIDE] §5.2), q/k RMSNorm across heads (R5), no RoPE."""
+    text context ([WAN21-GUIDE] §5.2), q/k RMSNorm across heads (R5), no RoPE.
+    With ``img`` (I2V, [B, Li, D] embedded image tokens) a second, separately
+    normalised attention over the image tokens is added before the output
+    projection ([WAN21-GUIDE] §4 table: the CLIP condition takes its own image
+    cross-attention; [ANIMATE-DIFF] "配置参数全解": an added key/value projection,
+    and its architecture section: image embeddings joined in front of the text
+    embeddings; reading R20)."""
     eps = cfg["eps"]
     q = rms_norm(linear(yc, Wb["attn2.to_q.weight"], Wb["attn2.to_q.bias"]), eps, Wb["attn2.norm_q.weight"])
     k = rms_norm(linear(ctx, Wb["attn2.to_k.weight"], Wb["attn2.to_k.bias"]), eps, Wb["attn2.norm_k.weight"])
     v = linear(ctx, Wb["attn2.to_v.weight"], Wb["attn2.to_v.bias"])
     o = attention(_heads(q, cfg), _heads(k, cfg), _heads(v, cfg)).reshape(q.shape)
+    if img is not None:
+        ki = rms_norm(linear(img, Wb["attn2.add_k_proj.weight"], Wb["attn2.add_k_proj.bias"]), eps,
+                      Wb["attn2.norm_added_k.weight"])
+        vi = linear(img, Wb["attn2.add_v_proj.weight"], Wb["attn2.add_v_proj.bias"])
+        o = o + attention(_heads(q, cfg), _heads(ki, cfg), _heads(vi, cfg)).reshape(q.shape)
     return linear(o, Wb["attn2.to_out.0.weight"], Wb["attn2.to_out.0.bias"])
 
 
@@ -342,14 +388,15 @@ def feed_forward(y, Wb):
     return linear(h, Wb["ffn.net.2.weight"], Wb["ffn.net.2.bias"])
 
 
-def block_forward(x, ctx, mod, Wb, angles, cfg, rows=None):
+def block_forward(x, ctx, mod, Wb, angles, cfg, rows=None, img=None):
     """One ``WanTransformerBlock`` ([PSWP-WAN] "WanTransformerBlock"; order also
     in [WAN21-GUIDE] §5.2).
 
     x [B, L, D]; ctx [B, Lc, D]; mod [B, 1 or L, 6, D] = block table + shared
     timestep projection, in the order shift, scale, gate, c_shift, c_scale,
     c_gate.  With ``rows`` (a LongTensor of token indices) only those tokens'
-    outputs are computed; keys and values still use every token.
+    outputs are computed; keys and values still use every token.  ``img``: the
+    embedded image tokens of the I2V route (R20), or None.
     """
     eps = cfg["eps"]
     shift, scale, gate, c_shift, c_scale, c_gate = (mod[:, :, n] for n in range(6))
@@ -363,7 +410,7 @@ def block_forward(x, ctx, mod, Wb, angles, cfg, rows=None):
     xr = xr + self_attention(y, Wb, angles, cfg, rows) * sel(gate)
     # 2. cross-attention after the affine norm2, plain residual
     yc = layer_norm(xr, eps, Wb["norm2.weight"], Wb["norm2.bias"])
-    xr = xr + cross_attention(yc, ctx, Wb, cfg)
+    xr = xr + cross_attention(yc, ctx, Wb, cfg, img)
     # 3. feed-forward with modulation and gated residual
     y = layer_norm(xr, eps) * (1.0 + sel(c_scale)) + sel(c_shift)
     return xr + feed_forward(y, Wb) * sel(c_gate)
@@ -386,7 +433,7 @@ def block_weights(W, i):
     return {k[len(p):]: v for k, v in W.items() if k.startswith(p)}
 
 
-def forward(latent, timestep, context, W, cfg, return_blocks: bool = False, rows=None):
+def forward(latent, timestep, context, W, cfg, return_blocks: bool = False, rows=None, image=None):
     """Velocity of one denoising step: patchify, conditioning, N blocks, head,
     unpatchify ([PSWP-WAN] "WanTransformer3DModel").
 
@@ -394,7 +441,10 @@ def forward(latent, timestep, context, W, cfg, return_blocks: bool = False, rows
     [B, Lc, text_dim].  Returns the velocity [B, C_out, F, Hz, Wz] and, with
     ``return_blocks``, the residual stream after the patch embedding and after
     every block.  With ``rows`` (one-block models only) the proj_out rows of
-    those tokens are returned instead of the velocity.
+    those tokens are returned instead of the velocity.  ``image`` (I2V): CLIP
+    tokens [B, Li, image_dim]; the forward listing of [PSWP-WAN] concatenates
+    the embedded image tokens before the text tokens and every block splits them
+    off again for the image attention (R20), so they are carried separately here.
     """
     B, C, F, Hz, Wz = latent.shape
     patch = tuple(cfg["patch"])
@@ -404,6 +454,7 @@ def forward(latent, timestep, context, W, cfg, return_blocks: bool = False, rows
     if tproj.dim() == 3:           # per-sample timestep: [B, 6, D] -> [B, 1, 6, D]
         tproj = tproj[:, None]
     ctx = text_embedding(context, W)
+    img = image_embedding(image, W) if image is not None else None
     angles = rope_angles(grid, cfg["rope_split"], cfg["rope_theta"])
     outs = [x] if return_blocks else None
     nb = cfg["num_blocks"]
@@ -412,7 +463,7 @@ def forward(latent, timestep, context, W, cfg, return_blocks: bool = False, rows
     for i in range(nb):
         Wb = block_weights(W, i)
         mod = Wb["scale_shift_table"].to(DT).reshape(1, 1, 6, cfg["dim"]) + tproj
-        x = block_forward(x, ctx, mod, Wb, angles, cfg, rows)
+        x = block_forward(x, ctx, mod, Wb, angles, cfg, rows, img)
         if return_blocks:
             outs.append(x)
     if rows is not None:
@@ -462,6 +513,16 @@ def param_shapes(cfg) -> Dict[str, Tuple[int, ...]]:
         s[p + "ffn.net.0.proj.bias"] = (Fd,)
         s[p + "ffn.net.2.weight"] = (D, Fd)
         s[p + "ffn.net.2.bias"] = (D,)
+        if cfg.get("image_dim", 0):
+            for n in ("add_k_proj", "add_v_proj"):
+                s[p + f"attn2.{n}.weight"] = (D, D)
+                s[p + f"attn2.{n}.bias"] = (D,)
+            s[p + "attn2.norm_added_k.weight"] = (D,)
+    if cfg.get("image_dim", 0):
+        s["condition_embedder.image_embedder.linear_1.weight"] = (D, cfg["image_dim"])
+        s["condition_embedder.image_embedder.linear_1.bias"] = (D,)
+        s["condition_embedder.image_embedder.linear_2.weight"] = (D, D)
+        s["condition_embedder.image_embedder.linear_2.bias"] = (D,)
     s["scale_shift_table"] = (1, 2, D)
     s["proj_out.weight"] = (Co * pt * ph * pw, D)
     s["proj_out.bias"] = (Co * pt * ph * pw,)
@@ -490,6 +551,17 @@ def flow_target(z, eps):
 def cfg_combine(v_uncond, v_cond, scale):
     """Classifier-free guidance v_u + s (v_c - v_u) ([WAN21-GUIDE] §7)."""
     return v_uncond + scale * (v_cond - v_uncond)
+
+
+def moe_expert(t: float, boundary: float, num_train_timesteps: int = 1000) -> int:
+    """Wan2.2 A14B expert for a sampling step: 0 = high-noise expert when
+    t >= boundary * num_train_timesteps, else 1 = low-noise expert.  One expert
+    serves a whole timestep, both CFG forwards included, and the switch compares
+    the scheduler's timestep value with boundary * num_train_timesteps
+    ([WAN22-PITFALLS] "一次生成会经过什么,又会在哪一步悄悄失败"); noise goes to the
+    high-noise expert first and to the low-noise one after the threshold
+    ([WAN21-GUIDE] §10.1).  Reading R21."""
+    return 0 if float(t) >= float(boundary) * num_train_timesteps else 1
 
 
 def euler_step(x, sigma, sigma_next, v):

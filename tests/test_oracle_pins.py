@@ -34,7 +34,7 @@ def rand_weights(cfg, seed=0, scale=0.3):
     W = {}
     for n, s in O.param_shapes(cfg).items():
         W[n] = torch.randn(*s, generator=g, dtype=DT) * scale
-        if ".norm_q." in n or ".norm_k." in n or n.endswith("norm2.weight"):
+        if ".norm_q." in n or ".norm_k." in n or n.endswith("norm2.weight") or ".norm_added_k." in n:
             W[n] = 1.0 + W[n]
     return W
 
@@ -313,7 +313,7 @@ def probe_setup(cfg, L=6, Lc=3, seed=3):
     g = torch.Generator().manual_seed(seed)
     W = {n: torch.zeros(*s, dtype=DT) for n, s in O.param_shapes(cfg).items()}
     for n in W:
-        if ".norm_q." in n or ".norm_k." in n or n.endswith("norm2.weight"):
+        if ".norm_q." in n or ".norm_k." in n or n.endswith("norm2.weight") or ".norm_added_k." in n:
             W[n] = torch.ones_like(W[n])
     D = cfg["dim"]
     x = torch.randn(1, L, D, generator=g, dtype=DT)
@@ -518,6 +518,115 @@ def test_row_sampling_matches_full_forward():
     vel = O.forward(lat, tt, ctx, W, cfg)
     o = O.forward(lat, tt, ctx, W, cfg, rows=rows)
     torch.testing.assert_close(o, vel.reshape(2, -1)[:, idx], rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- I2V route and MoE switch
+
+@pytest.mark.parametrize("case", GOLD["i2v"]["input_channels"], ids=lambda c: str(c["z_dim"]))
+def test_i2v_input_is_a_channel_concat(case):
+    z, m = case["z_dim"], case["mask_channels"]
+    g = torch.Generator().manual_seed(20)
+    noisy = torch.randn(1, z, 3, 4, 4, generator=g, dtype=DT)
+    cond = torch.randn(1, z, 3, 4, 4, generator=g, dtype=DT)
+    mask = torch.randn(1, m, 3, 4, 4, generator=g, dtype=DT)
+    x = O.i2v_input(noisy, cond, mask)
+    assert x.shape == (1, case["in_ch"], 3, 4, 4)          # channel axis, frames unchanged
+    assert torch.equal(x[:, :z], noisy) and torch.equal(x[:, z:2 * z], cond) and torch.equal(x[:, 2 * z:], mask)
+    with pytest.raises(ValueError):
+        O.i2v_input(noisy, cond, mask[:, :, :2])             # the mask must cover the same frames
+
+
+def test_i2v_patch_features_and_image_table():
+    pi, it = GOLD["i2v"]["patch_in"], GOLD["i2v"]["image_tokens"]
+    cfg = configs.model_config("wan2.1-i2v-14b")
+    assert cfg["in_ch"] * math.prod(cfg["patch"]) == pi["features"] and cfg["dim"] == pi["dim"]
+    assert cfg["image_dim"] == it["width"]
+    shapes = O.param_shapes(cfg)
+    assert shapes["patch_embedding.weight"] == (pi["dim"], pi["in_ch"], *pi["patch"])
+    assert shapes["condition_embedder.image_embedder.linear_1.weight"] == (cfg["dim"], it["width"])
+    # the image branch adds exactly its embedder and two projections + one gain per block
+    extra = O.param_count(cfg) - O.param_count(dict(cfg, image_dim=0, in_ch=36))
+    D = cfg["dim"]
+    assert extra == D * it["width"] + D + D * D + D + cfg["num_blocks"] * (2 * (D * D + D) + D)
+
+
+def i2v_tiny():
+    cfg = tiny_cfg(num_blocks=2, in_ch=9, image_dim=10)
+    W = rand_weights(cfg, seed=21)
+    g = torch.Generator().manual_seed(22)
+    lat = torch.randn(2, 9, 2, 4, 6, generator=g, dtype=DT)
+    ctx = torch.randn(2, 3, cfg["text_dim"], generator=g, dtype=DT)
+    img = torch.randn(2, 5, 10, generator=g, dtype=DT)
+    t = torch.full((2,), 700.0, dtype=DT)
+    return cfg, W, lat, t, ctx, img
+
+
+def test_i2v_image_branch_is_additive():
+    """With the image value projection at zero the image attention outputs zero, so
+    the I2V forward equals the forward without image tokens (same other weights)."""
+    cfg, W, lat, t, ctx, img = i2v_tiny()
+    v_img = O.forward(lat, t, ctx, W, cfg, image=img)
+    v_txt = O.forward(lat, t, ctx, W, cfg)
+    assert (v_img - v_txt).abs().max() > 1e-3                # the branch does something
+    for i in range(2):
+        W[f"blocks.{i}.attn2.add_v_proj.weight"].zero_()
+        W[f"blocks.{i}.attn2.add_v_proj.bias"].zero_()
+    torch.testing.assert_close(O.forward(lat, t, ctx, W, cfg, image=img), v_txt, rtol=1e-12, atol=1e-13)
+
+
+def test_i2v_single_image_token_closed_form():
+    """One image token: its softmax weight is 1, so the image attention returns its
+    value row for every query; the block output follows by hand."""
+    cfg, W, lat, t, ctx, img = i2v_tiny()
+    Wb = O.block_weights(W, 0)
+    g = torch.Generator().manual_seed(23)
+    yc = torch.randn(2, 7, cfg["dim"], generator=g, dtype=DT)
+    ctx_e = O.text_embedding(ctx, W)
+    img_e = O.image_embedding(img[:, :1], W)
+    got = O.cross_attention(yc, ctx_e, Wb, cfg, img_e)
+    eps = cfg["eps"]
+    q = O.rms_norm(O.linear(yc, Wb["attn2.to_q.weight"], Wb["attn2.to_q.bias"]), eps, Wb["attn2.norm_q.weight"])
+    k = O.rms_norm(O.linear(ctx_e, Wb["attn2.to_k.weight"], Wb["attn2.to_k.bias"]), eps, Wb["attn2.norm_k.weight"])
+    v = O.linear(ctx_e, Wb["attn2.to_v.weight"], Wb["attn2.to_v.bias"])
+    hq = lambda z: z.reshape(z.shape[0], z.shape[1], cfg["heads"], cfg["head_dim"]).transpose(1, 2)
+    o_txt = Fn.scaled_dot_product_attention(hq(q), hq(k), hq(v)).transpose(1, 2).reshape(q.shape)
+    vi = O.linear(img_e, Wb["attn2.add_v_proj.weight"], Wb["attn2.add_v_proj.bias"])   # [2, 1, D]
+    ref = O.linear(o_txt + vi, Wb["attn2.to_out.0.weight"], Wb["attn2.to_out.0.bias"])
+    torch.testing.assert_close(got, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_i2v_image_tokens_carry_no_order_and_are_per_sample():
+    cfg, W, lat, t, ctx, img = i2v_tiny()
+    v = O.forward(lat, t, ctx, W, cfg, image=img)
+    torch.testing.assert_close(O.forward(lat, t, ctx, W, cfg, image=img[:, [4, 2, 0, 1, 3]]), v,
+                               rtol=1e-11, atol=1e-12)
+    # sample 1's image does not reach sample 0
+    img2 = img.clone()
+    img2[1] = torch.randn(5, 10, dtype=DT)
+    v2 = O.forward(lat, t, ctx, W, cfg, image=img2)
+    torch.testing.assert_close(v2[0], v[0], rtol=0, atol=0)
+    assert (v2[1] - v[1]).abs().max() > 1e-6
+
+
+def test_image_embedding_is_two_linears_around_gelu():
+    cfg, W, lat, t, ctx, img = i2v_tiny()
+    p = "condition_embedder.image_embedder."
+    h = Fn.linear(img, W[p + "linear_1.weight"], W[p + "linear_1.bias"])
+    ref = Fn.linear(Fn.gelu(h, approximate="tanh"), W[p + "linear_2.weight"], W[p + "linear_2.bias"])
+    torch.testing.assert_close(O.image_embedding(img, W), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_moe_expert_switch():
+    assert "boundary * num_train_timesteps" in GOLD["moe_switch"]["rule"]
+    # a sampling schedule runs t downwards: the high-noise expert first, then the low-noise one, never back
+    ts = torch.linspace(999, 0, 50)
+    experts = [O.moe_expert(float(t), 0.875) for t in ts]
+    assert experts[0] == 0 and experts[-1] == 1
+    assert experts == sorted(experts)                       # one switch, high -> low
+    assert O.moe_expert(875.0, 0.875) == 0                  # the comparison includes the boundary
+    assert O.moe_expert(874.999, 0.875) == 1
+    assert O.moe_expert(900.0, 0.9, 1000) == 0 and O.moe_expert(899.0, 0.9, 1000) == 1
+    assert O.moe_expert(90.0, 0.9, 100) == 0                # scales with num_train_timesteps
 
 
 # ---------------------------------------------------------------- sizes and generator table

@@ -59,6 +59,15 @@ def param_shapes(cfg) -> Dict[str, Tuple[int, ...]]:
         s[p + "ffn.net.0.proj.bias"] = (Fd,)
         s[p + "ffn.net.2.weight"] = (D, Fd)
         s[p + "ffn.net.2.bias"] = (D,)
+        if cfg.get("image_dim", 0):  # image branch of the cross-attention (I2V)
+            for n in ("add_k_proj", "add_v_proj"):
+                s[p + f"attn2.{n}.weight"] = (D, D)
+                s[p + f"attn2.{n}.bias"] = (D,)
+            s[p + "attn2.norm_added_k.weight"] = (D,)
+    if cfg.get("image_dim", 0):
+        for n, (o, i) in (("image_embedder.linear_1", (D, cfg["image_dim"])), ("image_embedder.linear_2", (D, D))):
+            s[ce + n + ".weight"] = (o, i)
+            s[ce + n + ".bias"] = (o,)
     s["scale_shift_table"] = (1, 2, D)
     s["proj_out.weight"] = (Co * pt * ph * pw, D)
     s["proj_out.bias"] = (Co * pt * ph * pw,)
@@ -68,7 +77,7 @@ def param_shapes(cfg) -> Dict[str, Tuple[int, ...]]:
 def weight_kind(name: str) -> str:
     if name.endswith("scale_shift_table"):
         return "table"
-    if ".norm_q." in name or ".norm_k." in name or ".norm2.weight" in name:
+    if ".norm_q." in name or ".norm_k." in name or ".norm2.weight" in name or ".norm_added_k." in name:
         return "gain"
     if ".norm2.bias" in name:
         return "fp32bias"
@@ -112,6 +121,11 @@ def make_latent(shape, seed=0, device="cpu", same_across_batch=False) -> torch.T
 def make_context(B, Lc, text_dim, seed=0, device="cpu") -> torch.Tensor:
     """Text context [B, Lc, text_dim] bf16 of N(0, 1) (stands in for umT5 output)."""
     return _randn((B, Lc, text_dim), seed, "context", device).to(torch.bfloat16)
+
+
+def make_image(B, Li, image_dim, seed=0, device="cpu") -> torch.Tensor:
+    """Image tokens [B, Li, image_dim] bf16 of N(0, 1) (stands in for CLIP output)."""
+    return _randn((B, Li, image_dim), seed, "image", device).to(torch.bfloat16)
 
 
 def make_timestep(B, value) -> torch.Tensor:
