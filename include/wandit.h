@@ -73,14 +73,20 @@ enum { WAN_DTYPE_F32 = 0, WAN_DTYPE_BF16 = 1 };
  *   head_dim   must be 128 (attention_head_dim of every Wan model)
  *   ffn_dim    FFN hidden width (multiple of 64)
  *   num_blocks number of WanTransformerBlocks (30 for 1.3B/5B, 40 for 14B)
- *   in_ch/out_ch latent channels (16 for the Wan2.1 VAE, 48 for Wan2.2-5B)
+ *   in_ch/out_ch latent channels in and out (16 for the Wan2.1 VAE, 48 for
+ *              Wan2.2-5B; in_ch 36 = 16 noisy + 16 condition + 4 mask channels
+ *              for the I2V route, "I2V分量" table of the Wan2.1 source guide)
  *   patch_t/h/w patch size; only (1,2,2) is supported
  *   text_dim   context width (4096, umT5), multiple of 64
  *   freq_dim   timestep sinusoid width (256)
  *   rope_t/h/w head-dim split of the 3-axis RoPE (44/42/42), even, sum = head_dim
  *   eps        LayerNorm / RMSNorm epsilon (1e-6)
  *   rope_theta RoPE base (1e4)
- *   max_batch, max_tokens, max_text   workspace limits fixed at create      */
+ *   max_batch, max_tokens, max_text   workspace limits fixed at create
+ *   image_dim  width of the image (CLIP) tokens of the I2V route (1280), a
+ *              multiple of 64; 0 = no image branch (text-to-video models)
+ *   max_image  workspace limit on image tokens per sample (257 for CLIP);
+ *              ignored when image_dim is 0                                  */
 typedef struct {
     int dim, heads, head_dim, ffn_dim, num_blocks;
     int in_ch, out_ch, patch_t, patch_h, patch_w;
@@ -88,6 +94,7 @@ typedef struct {
     int rope_t, rope_h, rope_w;
     float eps, rope_theta;
     int max_batch, max_tokens, max_text;
+    int image_dim, max_image;
 } wan_dit_config;
 
 /* Create a handle on CUDA device `device` and allocate its workspace for
@@ -133,6 +140,34 @@ WANDIT_API wan_status wan_dit_forward(wan_dit* h, const void* latent, int latent
                            const void* context, int Lc,
                            float* velocity, int io_on_device, void* stream);
 
+/* The I2V forward (Wan2.1-I2V / Wan2.2-I2V route): as wan_dit_forward, with
+ *   latent    [B, in_ch, F, Hz, Wz], in_ch = 36 for the I2V models: noisy
+ *             latent, first-frame condition latent and known-frame mask joined
+ *             on the channel axis
+ *   image     bf16 [B, Li, image_dim] image tokens (CLIP, Li = 257), device or
+ *             host pointer like the other buffers; 1 <= Li <= max_image
+ * The image tokens pass the image embedder (two linears around GELU_tanh) and,
+ * in every block, a separate attention with their own key/value projections
+ * (blocks.{i}.attn2.add_k_proj / add_v_proj, keys RMSNorm'd across heads with
+ * attn2.norm_added_k) whose output is added to the text attention output
+ * before attn2.to_out (the model forward of the diffusers notes joins the
+ * image tokens in front of the text tokens; the Wan2.1 guide's §4 gives the
+ * CLIP condition its own image cross-attention).  image == NULL runs the text
+ * branch alone.  WAN_EINVAL if the model has no image branch (image_dim 0). */
+WANDIT_API wan_status wan_dit_forward_image(wan_dit* h, const void* latent, int latent_dtype,
+                           int B, int F, int Hz, int Wz,
+                           const float* timestep, int per_token,
+                           const void* context, int Lc,
+                           const void* image, int Li,
+                           float* velocity, int io_on_device, void* stream);
+
+/* Expert of the Wan2.2 A14B two-expert route for one sampling step: 0 (the
+ * high-noise expert) when t >= boundary * num_train_timesteps, else 1 (the
+ * low-noise expert).  One expert runs the whole step, both CFG forwards
+ * included ("读完 Wan2.2 全部源码之后", the sampling-loop section); the caller
+ * keeps one handle per expert.  Pure host function.                         */
+WANDIT_API int wan_moe_select(double t, double boundary, int num_train_timesteps);
+
 /* Synchronise `stream` and report a kernel timeout recorded by any earlier
  * launch of this handle (WAN_ETIMEOUT, flag cleared) or a CUDA error.       */
 WANDIT_API wan_status wan_dit_sync(wan_dit* h, void* stream);
@@ -167,6 +202,8 @@ WANDIT_API int wan_dit_last_launch_count(const wan_dit* h);
 
 /* Algorithmic FLOPs of one forward at the given shape (dense, no padding). */
 WANDIT_API double wan_dit_flops(const wan_dit* h, int B, int F, int Hz, int Wz, int Lc, int per_token);
+/* Same with Li image tokens per sample (I2V); Li = 0 equals wan_dit_flops. */
+WANDIT_API double wan_dit_flops_image(const wan_dit* h, int B, int F, int Hz, int Wz, int Lc, int per_token, int Li);
 
 WANDIT_API const char* wan_dit_last_error(const wan_dit* h);
 WANDIT_API const char* wan_status_string(wan_status s);

@@ -50,12 +50,28 @@ def test_create_rejects_unsupported_configs_without_a_device(lib):
         h = ctypes.c_void_p()
         assert lib.wan_dit_create(ctypes.byref(c), 0, ctypes.byref(h)) == 10   # WAN_EUNSUPPORTED
         assert not h
+    # image branch: width a multiple of 64, and a token limit with it
+    i2v = configs.model_config("wan2.1-i2v-14b")
+    for cfg, max_image in ((dict(i2v, image_dim=1000), 257), (i2v, 0)):
+        c = binding.make_config(cfg, 1, 192, 32, max_image)
+        h = ctypes.c_void_p()
+        assert lib.wan_dit_create(ctypes.byref(c), 0, ctypes.byref(h)) == 10
+        assert not h
     h = ctypes.c_void_p()
     assert lib.wan_dit_create(None, 0, ctypes.byref(h)) == 1                   # WAN_EINVAL
 
 
+def test_moe_select_follows_the_switch_rule(lib):
+    from oracle import wan_oracle as O
+    from video_diffusion_transformer_dit_b200 import binding
+    for boundary, n in ((0.875, 1000), (0.9, 1000), (0.5, 100)):
+        for t in [0.0, 1.0, 87.4, 87.5, 450.0, 874.999, 875.0, 875.001, 899.9, 900.0, 999.0]:
+            assert binding.moe_select(t, boundary, n) == O.moe_expert(t, boundary, n), (t, boundary, n)
+
+
 def test_null_handle_calls_are_refused(lib):
     assert lib.wan_dit_forward(None, None, 0, 1, 1, 2, 2, None, 0, None, 1, None, 1, None) == 1
+    assert lib.wan_dit_forward_image(None, None, 0, 1, 1, 2, 2, None, 0, None, 1, None, 0, None, 1, None) == 1
     assert lib.wan_dit_sync(None, None) == 1
     assert lib.wan_dit_last_launch_count(None) == 0
     assert lib.wan_dit_last_error(None) == b"null handle"

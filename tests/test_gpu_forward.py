@@ -218,3 +218,85 @@ def test_forward_33f_352x640_all_30_blocks_full_oracle():
     print(f"velocity rel-L2 {err:.3e}")
     assert max(errs) < TOL
     assert err < TOL
+
+
+# ---------------------------------------------------------------- I2V route and the expert switch
+
+def _i2v_case(seed=0):
+    from video_diffusion_transformer_dit_b200 import configs, synth
+    w = configs.workload("wan-i2v-1blk-3x16x16")
+    cfg = w["cfg"]
+    B, Cc, F, Hz, Wz = w["latent"]
+    W = synth.make_weights(cfg, seed=seed)
+    lat = synth.make_latent(w["latent"], seed=seed)
+    ctx = synth.make_context(B, w["text_len"], cfg["text_dim"], seed=seed)
+    img = synth.make_image(B, w["image_len"], cfg["image_dim"], seed=seed)
+    t = synth.make_timestep(B, w["timesteps"][0])
+    return cfg, W, lat, t, ctx, img
+
+
+def test_forward_i2v_one_block_against_oracle():
+    """36-channel input (patch K 144, padded to the 64-wide K tile), 257 image
+    tokens of width 1280 per sample, B = 2 with different images."""
+    from video_diffusion_transformer_dit_b200.binding import WanDiT
+    cfg, W, lat, t, ctx, img = _i2v_case()
+    B, L, Lc, Li = lat.shape[0], O.token_count(*lat.shape[2:]), ctx.shape[1], img.shape[1]
+    dit = WanDiT(cfg, max_batch=B, max_tokens=L, max_text=Lc, max_image=Li)
+    dit.load_weights({k: v.cuda() for k, v in W.items()})
+    assert dit.missing_weights()[0] == 0
+    v = dit.forward(lat.cuda(), t.cuda(), ctx.cuda(), image=img.cuda(), sync=True).cpu()
+    W64 = to64(W)
+    ref = O.forward(lat.to(DT), t.to(DT), ctx.to(DT), W64, cfg, image=img.to(DT))
+    err = rel_l2(v, ref)
+    print(f"\n[I2V 1 block] velocity rel-L2 {err:.3e}")
+    assert err < TOL
+    # the image branch matters, and without image tokens the text branch alone runs
+    v_txt = dit.forward(lat.cuda(), t.cuda(), ctx.cuda(), sync=True).cpu()
+    ref_txt = O.forward(lat.to(DT), t.to(DT), ctx.to(DT), W64, cfg)
+    assert rel_l2(v_txt, ref_txt) < TOL
+    assert rel_l2(ref, ref_txt) > 5 * TOL             # ~0.26 for these synthetic weights
+    # graph replay of the image plan is deterministic, host I/O equals device I/O
+    v2 = dit.forward(lat.cuda(), t.cuda(), ctx.cuda(), image=img.cuda(), sync=True).cpu()
+    assert torch.equal(v, v2)
+    v_host = dit.forward(lat.pin_memory(), t.pin_memory(), ctx.pin_memory(), image=img.pin_memory())
+    dit.sync()
+    assert torch.equal(v_host, v)
+    assert dit.flops(B, *lat.shape[2:], Lc, 0, Li) > dit.flops(B, *lat.shape[2:], Lc, 0)
+
+
+def test_forward_image_argument_validation():
+    from video_diffusion_transformer_dit_b200.binding import WanError
+    cfg, W, lat, t, ctx, img = _i2v_case(seed=1)
+    B, L, Lc = lat.shape[0], O.token_count(*lat.shape[2:]), ctx.shape[1]
+    from video_diffusion_transformer_dit_b200.binding import WanDiT
+    dit = WanDiT(cfg, max_batch=B, max_tokens=L, max_text=Lc, max_image=100)
+    dit.load_weights({k: v.cuda() for k, v in W.items()})
+    with pytest.raises(WanError) as e:                      # more image tokens than the workspace holds
+        dit.forward(lat.cuda(), t.cuda(), ctx.cuda(), image=img.cuda())
+    assert e.value.name == "WAN_ESHAPE"
+    t2v_cfg, W2, lat2, t2, ctx2 = workload_inputs("wan1.3b-1blk-3x16x16")
+    t2v = make_dit(t2v_cfg, 1, O.token_count(*lat2.shape[2:]), ctx2.shape[1], W2)
+    with pytest.raises(WanError) as e:                      # a text-to-video model has no image branch
+        t2v.forward(lat2.cuda(), t2.cuda(), ctx2.cuda(), image=img[:1, :10].cuda())
+    assert e.value.name == "WAN_EINVAL"
+
+
+def test_moe_expert_dispatch():
+    """Two handles with different weights: each step runs on the expert its
+    timestep selects, bit-identical to calling that expert directly."""
+    from video_diffusion_transformer_dit_b200 import synth
+    from video_diffusion_transformer_dit_b200.binding import WanMoE
+    cfg, W_hi, lat, t, ctx = workload_inputs("wan1.3b-1blk-3x16x16", seed=4)
+    W_lo = synth.make_weights(cfg, seed=5)
+    L, Lc = O.token_count(*lat.shape[2:]), ctx.shape[1]
+    hi, lo = make_dit(cfg, 1, L, Lc, W_hi), make_dit(cfg, 1, L, Lc, W_lo)
+    moe = WanMoE(hi, lo, boundary=0.875, num_train_timesteps=1000)
+    for tv, which in ((999.0, hi), (875.0, hi), (874.0, lo), (20.0, lo)):
+        tt = torch.full((1,), tv)
+        got = moe.forward(lat.cuda(), tt.cuda(), ctx.cuda(), sync=True).cpu()
+        want = which.forward(lat.cuda(), tt.cuda(), ctx.cuda(), sync=True).cpu()
+        assert torch.equal(got, want), tv
+    ref_lo = O.forward(lat.to(DT), torch.full((1,), 20.0, dtype=DT), ctx.to(DT), to64(W_lo), cfg)
+    assert rel_l2(moe.forward(lat.cuda(), torch.full((1,), 20.0).cuda(), ctx.cuda(), sync=True).cpu(), ref_lo) < TOL
+    with pytest.raises(ValueError):                           # one timestep per step
+        moe.expert(torch.tensor([900.0, 100.0]))

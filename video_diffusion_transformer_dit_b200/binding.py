@@ -27,7 +27,7 @@ EPI = {"bias": 0, "bias_gelu": 1, "gate_residual": 2, "residual": 3, "bias_f32":
 # every symbol include/*.h declares
 SYMBOLS = ["wan_dit_create", "wan_dit_load_weights", "wan_dit_missing_weights", "wan_dit_forward", "wan_dit_sync",
            "wan_dit_set_block_dump", "wan_dit_set_option", "wan_dit_kernel_time", "wan_dit_last_launch_count",
-           "wan_dit_flops",
+           "wan_dit_flops", "wan_dit_forward_image", "wan_dit_flops_image", "wan_moe_select",
            "wan_dit_last_error", "wan_status_string", "wan_dit_destroy",
            "wan_op_gemm", "wan_op_attention", "wan_op_layernorm", "wan_op_rmsnorm_rope", "wan_op_patchify",
            "wan_op_unpatchify", "wan_op_sync", "wan_op_set_wait_limit_ns", "wan_op_rmsnorm_rope_noalloc", "wan_op_cfg_euler",
@@ -46,7 +46,7 @@ class wan_dit_config(C.Structure):
                                         "patch_t", "patch_h", "patch_w", "text_dim", "freq_dim",
                                         "rope_t", "rope_h", "rope_w")] + \
               [("eps", C.c_float), ("rope_theta", C.c_float)] + \
-              [(n, C.c_int) for n in ("max_batch", "max_tokens", "max_text")]
+              [(n, C.c_int) for n in ("max_batch", "max_tokens", "max_text", "image_dim", "max_image")]
 
 
 class wan_epilogue(C.Structure):
@@ -80,6 +80,9 @@ def lib() -> C.CDLL:
         "wan_dit_kernel_time": (I, [P, I, C.POINTER(D), C.POINTER(I)]),
         "wan_dit_last_launch_count": (I, [P]),
         "wan_dit_flops": (D, [P, I, I, I, I, I, I]),
+        "wan_dit_forward_image": (I, [P, P, I, I, I, I, I, P, I, P, I, P, I, P, I, P]),
+        "wan_dit_flops_image": (D, [P, I, I, I, I, I, I, I]),
+        "wan_moe_select": (I, [D, D, I]),
         "wan_dit_last_error": (C.c_char_p, [P]),
         "wan_status_string": (C.c_char_p, [I]),
         "wan_dit_destroy": (None, [P]),
@@ -128,7 +131,7 @@ def _dtype_code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def make_config(cfg: dict, max_batch: int, max_tokens: int, max_text: int) -> wan_dit_config:
+def make_config(cfg: dict, max_batch: int, max_tokens: int, max_text: int, max_image: int = 0) -> wan_dit_config:
     c = wan_dit_config()
     for k in ("dim", "heads", "head_dim", "ffn_dim", "num_blocks", "in_ch", "out_ch", "text_dim", "freq_dim"):
         setattr(c, k, int(cfg[k]))
@@ -137,16 +140,19 @@ def make_config(cfg: dict, max_batch: int, max_tokens: int, max_text: int) -> wa
     c.eps = float(cfg["eps"])
     c.rope_theta = float(cfg["rope_theta"])
     c.max_batch, c.max_tokens, c.max_text = int(max_batch), int(max_tokens), int(max_text)
+    c.image_dim = int(cfg.get("image_dim", 0))
+    c.max_image = int(max_image) if c.image_dim else 0
     return c
 
 
 class WanDiT:
     """Handle of ``wan_dit``: create / load_weights / forward / sync / destroy."""
 
-    def __init__(self, cfg: dict, max_batch: int, max_tokens: int, max_text: int, device: int = 0):
+    def __init__(self, cfg: dict, max_batch: int, max_tokens: int, max_text: int, device: int = 0,
+                 max_image: int = 257):
         self.cfg = dict(cfg)
         self._h = C.c_void_p()
-        c = make_config(cfg, max_batch, max_tokens, max_text)
+        c = make_config(cfg, max_batch, max_tokens, max_text, max_image)
         _check(lib().wan_dit_create(C.byref(c), int(device), C.byref(self._h)), "wan_dit_create")
 
     # -- lifetime
@@ -194,10 +200,11 @@ class WanDiT:
         return n, buf.value.decode()
 
     # -- forward
-    def forward(self, latent, timestep, context, velocity=None, stream=None, sync=False):
+    def forward(self, latent, timestep, context, velocity=None, stream=None, sync=False, image=None):
         """latent [B,C,F,Hz,Wz] f32/bf16, timestep f32 [B] or [B,L], context bf16
-        [B,Lc,text_dim].  All CUDA tensors (device I/O) or all CPU tensors (host
-        I/O, copies inside the call).  Returns the velocity tensor."""
+        [B,Lc,text_dim], image (I2V models) bf16 [B,Li,image_dim] or None.  All
+        CUDA tensors (device I/O) or all CPU tensors (host I/O, copies inside the
+        call).  Returns the velocity tensor."""
         import torch
         B, Cin, F, Hz, Wz = latent.shape
         Lc = context.shape[1]
@@ -207,8 +214,14 @@ class WanDiT:
             velocity = torch.empty(B, self.cfg["out_ch"], F, Hz, Wz, dtype=torch.float32, device=latent.device,
                                    pin_memory=not on_dev)
         st = _stream(stream)
-        self._check(lib().wan_dit_forward(self._h, _ptr(latent), _dtype_code(latent), B, F, Hz, Wz, _ptr(timestep),
-                                          per_token, _ptr(context), Lc, _ptr(velocity), int(on_dev), st))
+        if image is None:
+            self._check(lib().wan_dit_forward(self._h, _ptr(latent), _dtype_code(latent), B, F, Hz, Wz,
+                                              _ptr(timestep), per_token, _ptr(context), Lc, _ptr(velocity),
+                                              int(on_dev), st))
+        else:
+            self._check(lib().wan_dit_forward_image(self._h, _ptr(latent), _dtype_code(latent), B, F, Hz, Wz,
+                                                    _ptr(timestep), per_token, _ptr(context), Lc, _ptr(image),
+                                                    image.shape[1], _ptr(velocity), int(on_dev), st))
         if sync:
             self.sync(stream)
         return velocity
@@ -231,8 +244,34 @@ class WanDiT:
     def last_launch_count(self) -> int:
         return lib().wan_dit_last_launch_count(self._h)
 
-    def flops(self, B, F, Hz, Wz, Lc, per_token=0) -> float:
-        return lib().wan_dit_flops(self._h, B, F, Hz, Wz, Lc, per_token)
+    def flops(self, B, F, Hz, Wz, Lc, per_token=0, Li=0) -> float:
+        return lib().wan_dit_flops_image(self._h, B, F, Hz, Wz, Lc, per_token, Li)
+
+
+def moe_select(t: float, boundary: float, num_train_timesteps: int = 1000) -> int:
+    """0 (high-noise expert) when t >= boundary * num_train_timesteps, else 1."""
+    return lib().wan_moe_select(float(t), float(boundary), int(num_train_timesteps))
+
+
+class WanMoE:
+    """Two-expert route (Wan2.2 A14B): one ``WanDiT`` handle per expert and the
+    timestep switch of ``wan_moe_select``; a step's forwards (both CFG branches)
+    all run on the expert its timestep selects."""
+
+    def __init__(self, high_noise: WanDiT, low_noise: WanDiT, boundary: float, num_train_timesteps: int = 1000):
+        self.experts = (high_noise, low_noise)
+        self.boundary = float(boundary)
+        self.num_train_timesteps = int(num_train_timesteps)
+
+    def expert(self, timestep) -> int:
+        """Expert index of a per-sample timestep tensor [B] (all entries equal)."""
+        t = timestep.detach().float().cpu()
+        if t.dim() != 1 or not bool((t == t[0]).all()):
+            raise ValueError("the expert switch takes one per-sample timestep shared by the batch")
+        return moe_select(float(t[0]), self.boundary, self.num_train_timesteps)
+
+    def forward(self, latent, timestep, context, **kw):
+        return self.experts[self.expert(timestep)].forward(latent, timestep, context, **kw)
 
 
 # ---------------------------------------------------------------- op-level wrappers

@@ -341,41 +341,73 @@ cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float 
 
 // ------------------------------------------------------------------ patchify / unpatchify
 // X[b * L + (f * Hp + i) * Wp + j, c * 4 + kh * 2 + kw] = latent[b, c, f, 2i + kh, 2j + kw]
+// for c < C; columns [4C, ldx) of every row are written as zeros (K padding of
+// the patch GEMM when 4C is not a multiple of its K tile).
 template <typename T>
 __global__ void patchify_kernel(const T* __restrict__ lat, __nv_bfloat16* __restrict__ X, int B, int C, int F, int Hz,
-                                int Wz) {
+                                int Wz, int ldx) {
     const int Hp = Hz >> 1, Wp = Wz >> 1;
     const long long L = (long long)F * Hp * Wp;
-    const long long total = (long long)B * L * C;
+    const int G = ldx >> 2;  // groups of 4 columns per row
+    const long long total = (long long)B * L * G;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
-        const int c = idx % C;
-        const long long row = idx / C;
-        const int b = row / L;
-        const long long l = row - (long long)b * L;
-        const int f = l / (Hp * Wp);
-        const int rem = l - (long long)f * (Hp * Wp);
-        const int i = rem / Wp, j = rem - (rem / Wp) * Wp;
-        const T* src = lat + ((((long long)b * C + c) * F + f) * Hz + 2 * i) * Wz + 2 * j;
-        float a = (float)src[0], bb = (float)src[1], cc = (float)src[Wz], d = (float)src[Wz + 1];
-        uint2 u = make_uint2(pack_bf16(a, bb), pack_bf16(cc, d));
-        *reinterpret_cast<uint2*>(X + row * (4 * C) + 4 * c) = u;
+        const int c = idx % G;
+        const long long row = idx / G;
+        uint2 u = make_uint2(0u, 0u);
+        if (c < C) {
+            const int b = row / L;
+            const long long l = row - (long long)b * L;
+            const int f = l / (Hp * Wp);
+            const int rem = l - (long long)f * (Hp * Wp);
+            const int i = rem / Wp, j = rem - (rem / Wp) * Wp;
+            const T* src = lat + ((((long long)b * C + c) * F + f) * Hz + 2 * i) * Wz + 2 * j;
+            float a = (float)src[0], bb = (float)src[1], cc = (float)src[Wz], d = (float)src[Wz + 1];
+            u = make_uint2(pack_bf16(a, bb), pack_bf16(cc, d));
+        }
+        *reinterpret_cast<uint2*>(X + row * ldx + 4 * c) = u;
     }
 }
 
 cudaError_t launch_patchify(const void* latent, int latent_dtype, int B, int C, int F, int Hz, int Wz, void* X,
-                            const LaunchCtx& ctx) {
-    const long long total = (long long)B * F * (Hz / 2) * (Wz / 2) * C;
+                            int ldx, const LaunchCtx& ctx) {
+    if (ldx < 4 * C || ldx % 4) return cudaErrorInvalidValue;
+    const long long total = (long long)B * F * (Hz / 2) * (Wz / 2) * (ldx / 4);
     if (total <= 0) return cudaSuccess;
     int grid = (int)((total + 255) / 256);
     if (grid > ctx.num_sms * 16) grid = ctx.num_sms * 16;
     if (latent_dtype == 0)
         patchify_kernel<float><<<grid, 256, 0, ctx.stream>>>(reinterpret_cast<const float*>(latent),
-                                                              reinterpret_cast<__nv_bfloat16*>(X), B, C, F, Hz, Wz);
+                                                              reinterpret_cast<__nv_bfloat16*>(X), B, C, F, Hz, Wz,
+                                                              ldx);
     else
         patchify_kernel<__nv_bfloat16><<<grid, 256, 0, ctx.stream>>>(reinterpret_cast<const __nv_bfloat16*>(latent),
                                                                       reinterpret_cast<__nv_bfloat16*>(X), B, C, F, Hz,
-                                                                      Wz);
+                                                                      Wz, ldx);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ a += b (bf16, fp32 sum, one rounding)
+__global__ void add_bf16_kernel(__nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b, long long n8) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+        float x[8], y[8];
+        load8(a + i * 8, x);
+        load8(b + i * 8, y);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] += y[k];
+        store8(a + i * 8, x);
+    }
+}
+
+cudaError_t launch_add_bf16(void* a, const void* b, long long n, const LaunchCtx& ctx) {
+    if (n <= 0) return cudaSuccess;
+    if (n % 8 || ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15)) return cudaErrorInvalidValue;
+    const long long n8 = n / 8;
+    long long g = (n8 + 255) / 256;
+    if (g > ctx.num_sms * 16) g = ctx.num_sms * 16;
+    add_bf16_kernel<<<(int)g, 256, 0, ctx.stream>>>(reinterpret_cast<__nv_bfloat16*>(a),
+                                                   reinterpret_cast<const __nv_bfloat16*>(b), n8);
     if (ctx.launches) ++*ctx.launches;
     return cudaGetLastError();
 }

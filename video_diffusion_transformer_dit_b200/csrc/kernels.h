@@ -84,7 +84,9 @@ cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float 
                                 int rope_L, const LaunchCtx& ctx);
 
 cudaError_t launch_patchify(const void* latent, int latent_dtype, int B, int C, int F, int Hz, int Wz, void* X,
-                            const LaunchCtx& ctx);
+                            int ldx, const LaunchCtx& ctx);  // ldx >= 4C: row stride of X, pad columns zeroed
+// a[i] = bf16(a[i] + b[i]) for n bf16 values (n % 8 == 0, 16-byte aligned)
+cudaError_t launch_add_bf16(void* a, const void* b, long long n, const LaunchCtx& ctx);
 cudaError_t launch_unpatchify(const float* rows, int B, int C, int F, int Hz, int Wz, float* vel,
                               const LaunchCtx& ctx);
 

@@ -80,7 +80,7 @@ struct Plan {
     int timed_pairs = 0;        // pairs recorded by the most recent timed forward
 };
 
-using PlanKey = std::tuple<int, int, int, int, int, int, int>;
+using PlanKey = std::tuple<int, int, int, int, int, int, int, int>;
 
 }  // namespace
 
@@ -97,6 +97,11 @@ struct wan_dit {
     std::vector<BlockW> blocks;
     void *w_pe, *w_t1, *w_t2, *w_tp, *w_x1, *w_x2, *w_kv, *w_po;
     float *b_pe, *b_t1, *b_t2, *b_tp, *b_x1, *b_x2, *b_kv, *k2_gain, *sst_out, *b_po;
+    int Kp = 0;           // patch GEMM K: 4 * in_ch rounded up to the 64-wide K tile
+    void* w_pe_k;         // [D, Kp] patch weights as the GEMM reads them (== w_pe when Kp == 4 * in_ch)
+    // image branch (image_dim > 0): embedder, all blocks' image K/V projections and key gains
+    void *w_i1 = nullptr, *w_i2 = nullptr, *w_kvi = nullptr;
+    float *b_i1 = nullptr, *b_i2 = nullptr, *b_kvi = nullptr, *ki_gain = nullptr;
     float* sst_all;       // [N, 6, D] block tables, contiguous
     // workspace
     char* ws = nullptr;
@@ -106,6 +111,7 @@ struct wan_dit {
     float* t_stage;       // f32 [R]
     float* vel_stage;     // f32 [R * out_ch * 4]
     void *X, *x, *y, *qkv, *o, *qc, *u, *th, *ctx, *kv, *tsin, *tsilu;
+    void *img_stage = nullptr, *ih = nullptr, *ictx = nullptr, *kvi = nullptr, *o2 = nullptr;  // image branch
     float *temb, *tproj, *th32;
     float* modc;          // [N, max_batch, 6, D] per-sample modulation of every block
     int* d_err = nullptr;
@@ -149,7 +155,7 @@ bool valid_config(const wan_dit_config& c, std::string& why) {
     if (c.ffn_dim <= 0 || c.ffn_dim % 64) return bad("ffn_dim must be a positive multiple of 64");
     if (c.num_blocks <= 0) return bad("num_blocks must be positive");
     if (c.patch_t != 1 || c.patch_h != 2 || c.patch_w != 2) return bad("only patch (1,2,2) is supported");
-    if (c.in_ch <= 0 || (c.in_ch * 4) % 64) return bad("in_ch * 4 must be a multiple of 64");
+    if (c.in_ch <= 0 || c.in_ch > 1024) return bad("in_ch must be 1..1024");
     if (c.out_ch <= 0 || (c.out_ch * 4) % 64) return bad("out_ch * 4 must be a multiple of 64");
     if (c.text_dim <= 0 || c.text_dim % 64) return bad("text_dim must be a positive multiple of 64");
     if (c.freq_dim <= 0 || c.freq_dim % 16) return bad("freq_dim must be a positive multiple of 16");
@@ -158,6 +164,8 @@ bool valid_config(const wan_dit_config& c, std::string& why) {
     if (!(c.eps > 0.f) || !(c.rope_theta > 0.f)) return bad("eps and rope_theta must be positive");
     if (c.max_batch <= 0 || c.max_batch > 8 || c.max_tokens <= 0 || c.max_text <= 0)
         return bad("max_batch must be 1..8; max_tokens, max_text positive");
+    if (c.image_dim < 0 || c.image_dim % 64) return bad("image_dim must be 0 or a positive multiple of 64");
+    if (c.image_dim > 0 && c.max_image <= 0) return bad("max_image must be positive with an image branch");
     return true;
 }
 
@@ -170,10 +178,16 @@ void add_slot(wan_dit* h, const std::string& name, void* dst, int dt, std::vecto
 wan_status build_weights(wan_dit* h) {
     const auto& c = h->cfg;
     const long long D = c.dim, Fd = c.ffn_dim, N = c.num_blocks, P_in = c.in_ch * 4, P_out = c.out_ch * 4;
+    const long long Kp = (P_in + 63) / 64 * 64, Di = c.image_dim;
+    h->Kp = (int)Kp;
     // sizes in bytes
     size_t total = 0;
     auto sz = [&](long long n, int dt) { size_t b = align_up(n * (dt == WAN_DTYPE_BF16 ? 2 : 4), 256); total += b; return b; };
     sz(D * P_in, 1); sz(D, 0);
+    if (Kp != P_in) sz(D * Kp, 1);
+    if (Di > 0) {
+        sz(D * Di, 1); sz(D, 0); sz(D * D, 1); sz(D, 0); sz(N * 2 * D * D, 1); sz(N * 2 * D, 0); sz(N * D, 0);
+    }
     sz(D * c.freq_dim, 1); sz(D, 0); sz(D * D, 1); sz(D, 0); sz(6 * D * D, 1); sz(6 * D, 0);
     sz(D * c.text_dim, 1); sz(D, 0); sz(D * D, 1); sz(D, 0);
     sz(N * 2 * D * D, 1); sz(N * 2 * D, 0); sz(N * D, 0); sz(N * 6 * D, 0);
@@ -198,6 +212,7 @@ wan_status build_weights(wan_dit* h) {
     h->b_pe = (float*)take(D, 0);
     add_slot(h, "patch_embedding.weight", h->w_pe, 1, {D, c.in_ch, c.patch_t, c.patch_h, c.patch_w});
     add_slot(h, "patch_embedding.bias", h->b_pe, 0, {D});
+    h->w_pe_k = Kp != P_in ? take(D * Kp, 1) : h->w_pe;  // zero pad columns (arena is zeroed)
     const std::string ce = "condition_embedder.";
     h->w_t1 = take(D * c.freq_dim, 1); h->b_t1 = (float*)take(D, 0);
     h->w_t2 = take(D * D, 1); h->b_t2 = (float*)take(D, 0);
@@ -219,6 +234,17 @@ wan_status build_weights(wan_dit* h) {
     h->b_kv = (float*)take(N * 2 * D, 0);
     h->k2_gain = (float*)take(N * D, 0);
     h->sst_all = (float*)take(N * 6 * D, 0);
+    if (Di > 0) {
+        h->w_i1 = take(D * Di, 1); h->b_i1 = (float*)take(D, 0);
+        h->w_i2 = take(D * D, 1); h->b_i2 = (float*)take(D, 0);
+        h->w_kvi = take(N * 2 * D * D, 1);
+        h->b_kvi = (float*)take(N * 2 * D, 0);
+        h->ki_gain = (float*)take(N * D, 0);
+        add_slot(h, ce + "image_embedder.linear_1.weight", h->w_i1, 1, {D, Di});
+        add_slot(h, ce + "image_embedder.linear_1.bias", h->b_i1, 0, {D});
+        add_slot(h, ce + "image_embedder.linear_2.weight", h->w_i2, 1, {D, D});
+        add_slot(h, ce + "image_embedder.linear_2.bias", h->b_i2, 0, {D});
+    }
     h->blocks.resize(N);
     for (int i = 0; i < N; ++i) {
         BlockW& b = h->blocks[i];
@@ -259,6 +285,13 @@ wan_status build_weights(wan_dit* h) {
         add_slot(h, p + "attn2.to_out.0.bias", b.bo2, 0, {D});
         add_slot(h, p + "attn2.norm_q.weight", b.q2_gain, 0, {D});
         add_slot(h, p + "attn2.norm_k.weight", f4(h->k2_gain, (long long)i * D), 0, {D});
+        if (Di > 0) {  // image branch of attn2: K/V rows of all blocks in one matrix, like the text K/V
+            add_slot(h, p + "attn2.add_k_proj.weight", bf(h->w_kvi, (2LL * i) * D * D), 1, {D, D});
+            add_slot(h, p + "attn2.add_v_proj.weight", bf(h->w_kvi, (2LL * i + 1) * D * D), 1, {D, D});
+            add_slot(h, p + "attn2.add_k_proj.bias", f4(h->b_kvi, 2LL * i * D), 0, {D});
+            add_slot(h, p + "attn2.add_v_proj.bias", f4(h->b_kvi, (2LL * i + 1) * D), 0, {D});
+            add_slot(h, p + "attn2.norm_added_k.weight", f4(h->ki_gain, (long long)i * D), 0, {D});
+        }
         add_slot(h, p + "ffn.net.0.proj.weight", b.w1, 1, {Fd, D});
         add_slot(h, p + "ffn.net.0.proj.bias", b.b1, 0, {Fd});
         add_slot(h, p + "ffn.net.2.weight", b.w2, 1, {D, Fd});
@@ -278,12 +311,13 @@ wan_status build_workspace(wan_dit* h) {
     const long long R = (long long)c.max_batch * c.max_tokens;
     const long long Rc = (long long)c.max_batch * c.max_text;
     const long long D = c.dim, Fd = c.ffn_dim, N = c.num_blocks;
-    const long long Pin = c.in_ch * 4, Pout = c.out_ch * 4;
+    const long long Pin = c.in_ch * 4, Pout = c.out_ch * 4, Kp = h->Kp;
+    const long long Ri = c.image_dim > 0 ? (long long)c.max_batch * c.max_image : 0;
     struct Item { void** p; size_t bytes; };
     std::vector<Item> items = {
         {(void**)&h->lat_stage, (size_t)(R * Pin * 4)}, {&h->ctx_stage, (size_t)(Rc * c.text_dim * 2)},
         {(void**)&h->t_stage, (size_t)(R * 4)},        {(void**)&h->vel_stage, (size_t)(R * Pout * 4)},
-        {&h->X, (size_t)(R * Pin * 2)},                {&h->x, (size_t)(R * D * 2)},
+        {&h->X, (size_t)(R * Kp * 2)},                 {&h->x, (size_t)(R * D * 2)},
         {&h->y, (size_t)(R * D * 2)},                  {&h->qkv, (size_t)(R * 3 * D * 2)},
         {&h->o, (size_t)(R * D * 2)},                  {&h->qc, (size_t)(R * D * 2)},
         {&h->u, (size_t)(R * Fd * 2)},                 {&h->th, (size_t)(Rc * D * 2)},
@@ -293,6 +327,13 @@ wan_status build_workspace(wan_dit* h) {
         {(void**)&h->th32, (size_t)(R * D * 4)},
         {(void**)&h->modc, (size_t)((long long)N * c.max_batch * 6 * D * 4)},
     };
+    if (Ri > 0) {
+        items.push_back({&h->img_stage, (size_t)(Ri * c.image_dim * 2)});
+        items.push_back({&h->ih, (size_t)(Ri * D * 2)});
+        items.push_back({&h->ictx, (size_t)(Ri * D * 2)});
+        items.push_back({&h->kvi, (size_t)(Ri * N * 2 * D * 2)});
+        items.push_back({&h->o2, (size_t)(R * D * 2)});
+    }
     size_t total = 0;
     for (auto& it : items) total += align_up(it.bytes, 1024);
     if (cudaMalloc(&h->ws, total) != cudaSuccess) {
@@ -333,7 +374,7 @@ void rope_tables_host(const wan_dit_config& c, int Fp, int Hp, int Wp, std::vect
 }
 
 struct Shape {
-    int B, F, Hz, Wz, Lc, per_token, lat_dtype;
+    int B, F, Hz, Wz, Lc, per_token, lat_dtype, Li;  // Li: image tokens per sample, 0 without the image branch
     int L() const { return F * (Hz / 2) * (Wz / 2); }
 };
 
@@ -366,8 +407,8 @@ cudaError_t issue_forward(wan_dit* h, const Shape& s, const Plan& plan, const La
         return p;
     };
     // ---- patch embedding: gather + GEMM (K = in_ch * 4)
-    TRYK(WAN_KC_PATCHIFY, wan::launch_patchify(h->lat_stage, s.lat_dtype, B, c.in_ch, s.F, s.Hz, s.Wz, h->X, ctx));
-    TRYK(WAN_KC_GEMM, wan::launch_gemm(h->X, c.in_ch * 4, h->w_pe, c.in_ch * 4, R, D, c.in_ch * 4,
+    TRYK(WAN_KC_PATCHIFY, wan::launch_patchify(h->lat_stage, s.lat_dtype, B, c.in_ch, s.F, s.Hz, s.Wz, h->X, h->Kp, ctx));
+    TRYK(WAN_KC_GEMM, wan::launch_gemm(h->X, h->Kp, h->w_pe_k, h->Kp, R, D, h->Kp,
                          epi(wan::EPI_BIAS, h->b_pe, h->x, D), ctx));
     if (dump) TRY(cudaMemcpyAsync(h->dump, h->x, (size_t)R * D * 2, cudaMemcpyDeviceToDevice, ctx.stream));
     // ---- timestep embedding -> temb [B|R, D] f32, tproj [B|R, 6D] f32
@@ -394,6 +435,17 @@ cudaError_t issue_forward(wan_dit* h, const Shape& s, const Plan& plan, const La
     const long long ldkv = 2LL * N * D;
     TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ctx, D, h->w_kv, D, Rc, (int)ldkv, D, epi(wan::EPI_BIAS, h->b_kv, h->kv, ldkv), ctx));
     TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rmsnorm_rope(h->kv, ldkv, Rc, D, c.eps, h->k2_gain, D, N, 2LL * D, nullptr, 0, ctx));
+    // ---- image tokens (I2V): embedder (Linear, GELU_tanh, Linear), then every block's image K/V and key norm
+    const int Ri = B * s.Li;
+    if (s.Li > 0) {
+        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->img_stage, c.image_dim, h->w_i1, c.image_dim, Ri, D, c.image_dim,
+                             epi(wan::EPI_BIAS_GELU, h->b_i1, h->ih, D), ctx));
+        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ih, D, h->w_i2, D, Ri, D, D, epi(wan::EPI_BIAS, h->b_i2, h->ictx, D), ctx));
+        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ictx, D, h->w_kvi, D, Ri, (int)ldkv, D, epi(wan::EPI_BIAS, h->b_kvi, h->kvi, ldkv),
+                             ctx));
+        TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rmsnorm_rope(h->kvi, ldkv, Ri, D, c.eps, h->ki_gain, D, N, 2LL * D, nullptr, 0,
+                                                           ctx));
+    }
 
     char* qkv = reinterpret_cast<char*>(h->qkv);
     for (int i = 0; i < N; ++i) {
@@ -426,6 +478,12 @@ cudaError_t issue_forward(wan_dit* h, const Shape& s, const Plan& plan, const La
         TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rmsnorm_rope(h->qc, D, R, D, c.eps, w.q2_gain, D, 1, 0, nullptr, 0, ctx));
         const char* kvb = reinterpret_cast<const char*>(h->kv) + 2LL * (2LL * i * D);
         TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_attention(h->qc, D, kvb, ldkv, kvb + 2LL * D, ldkv, h->o, D, B, c.heads, L, Lc, ctx));
+        if (s.Li > 0) {  // image attention with the same queries, added before attn2.to_out
+            const char* kvib = reinterpret_cast<const char*>(h->kvi) + 2LL * (2LL * i * D);
+            TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_attention(h->qc, D, kvib, ldkv, kvib + 2LL * D, ldkv, h->o2, D, B,
+                                                               c.heads, L, s.Li, ctx));
+            TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_add_bf16(h->o, h->o2, (long long)R * D, ctx));
+        }
         TRYK(WAN_KC_GEMM, wan::launch_gemm(h->o, D, w.wo2, D, R, D, D, epi(wan::EPI_RESIDUAL, w.bo2, h->x, D), ctx));
         // 3. feed-forward: norm3 + modulation (shift row 3, scale row 4), GELU-tanh, gated residual (row 5)
         if (!s.per_token)
@@ -466,7 +524,7 @@ cudaError_t issue_forward(wan_dit* h, const Shape& s, const Plan& plan, const La
 }
 
 wan_status ensure_plan(wan_dit* h, const Shape& s, Plan** out) {
-    PlanKey key{s.B, s.F, s.Hz, s.Wz, s.Lc, s.per_token, s.lat_dtype};
+    PlanKey key{s.B, s.F, s.Hz, s.Wz, s.Lc, s.per_token, s.lat_dtype, s.Li};
     auto it = h->plans.find(key);
     if (it != h->plans.end()) {
         *out = &it->second;
@@ -635,6 +693,13 @@ wan_status wan_dit_load_weights(wan_dit* h, int n, const char* const* names, con
         if (!ptrs_on_device) WAN_CU(cudaStreamSynchronize(st), "weight upload");
         h->loaded.insert(names[i]);
     }
+    if (h->w_pe_k != h->w_pe && h->loaded.count("patch_embedding.weight")) {
+        // [D, 4 * in_ch] -> [D, Kp]; the pad columns stay zero
+        const size_t row = (size_t)h->cfg.in_ch * 4 * 2;
+        WAN_CU(cudaMemcpy2DAsync(h->w_pe_k, (size_t)h->Kp * 2, h->w_pe, row, row, h->cfg.dim, cudaMemcpyDeviceToDevice,
+                                 st),
+               "patch weight repack");
+    }
     WAN_CU(cudaStreamSynchronize(st), "weight load");
     if (tmp) cudaFree(tmp);
     return first;
@@ -687,6 +752,10 @@ wan_status wan_dit_set_option(wan_dit* h, int option, int64_t value) {
 }
 
 double wan_dit_flops(const wan_dit* h, int B, int F, int Hz, int Wz, int Lc, int per_token) {
+    return wan_dit_flops_image(h, B, F, Hz, Wz, Lc, per_token, 0);
+}
+
+double wan_dit_flops_image(const wan_dit* h, int B, int F, int Hz, int Wz, int Lc, int per_token, int Li) {
     if (!h) return 0.0;
     const auto& c = h->cfg;
     const double L = (double)F * (Hz / 2) * (Wz / 2), D = c.dim, Fd = c.ffn_dim, N = c.num_blocks;
@@ -694,14 +763,30 @@ double wan_dit_flops(const wan_dit* h, int B, int F, int Hz, int Wz, int Lc, int
     double per_block = 2 * L * D * 6 * D + 4 * L * D * Fd + 4 * (double)Lc * D * D + 4 * L * L * D + 4 * L * Lc * D;
     double f = N * per_block + 2 * L * D * Pin + 2 * L * D * Pout + 2.0 * Lc * (c.text_dim * D + D * D);
     f += per_token ? 2 * L * (c.freq_dim * D + 7 * D * D) : 2 * (c.freq_dim * D + 7 * D * D);
+    if (Li > 0 && c.image_dim > 0)  // image embedder, per block image K/V projections and image attention
+        f += 2.0 * Li * ((double)c.image_dim * D + D * D) + N * (4.0 * Li * D * D + 4.0 * L * Li * D);
     return B * f;
+}
+
+int wan_moe_select(double t, double boundary, int num_train_timesteps) {
+    return t >= boundary * (double)num_train_timesteps ? 0 : 1;
 }
 
 wan_status wan_dit_forward(wan_dit* h, const void* latent, int latent_dtype, int B, int F, int Hz, int Wz,
                            const float* timestep, int per_token, const void* context, int Lc, float* velocity,
                            int io_on_device, void* stream) {
+    return wan_dit_forward_image(h, latent, latent_dtype, B, F, Hz, Wz, timestep, per_token, context, Lc, nullptr, 0,
+                                 velocity, io_on_device, stream);
+}
+
+wan_status wan_dit_forward_image(wan_dit* h, const void* latent, int latent_dtype, int B, int F, int Hz, int Wz,
+                                 const float* timestep, int per_token, const void* context, int Lc, const void* image,
+                                 int Li, float* velocity, int io_on_device, void* stream) {
     if (!h) return WAN_EINVAL;
     if (!latent || !timestep || !context || !velocity) return fail(h, WAN_EINVAL, "null input or output pointer");
+    if (image && h->cfg.image_dim <= 0) return fail(h, WAN_EINVAL, "image tokens given to a model without an image branch");
+    if (!image) Li = 0;
+    if (image && (Li < 1 || Li > h->cfg.max_image)) return fail(h, WAN_ESHAPE, "image token count outside 1..max_image");
     if (latent_dtype != WAN_DTYPE_F32 && latent_dtype != WAN_DTYPE_BF16) return fail(h, WAN_EINVAL, "latent dtype");
     const auto& c = h->cfg;
     if (B < 1 || B > c.max_batch) return fail(h, WAN_ESHAPE, "batch outside 1..max_batch");
@@ -718,7 +803,7 @@ wan_status wan_dit_forward(wan_dit* h, const void* latent, int latent_dtype, int
     }
     cudaSetDevice(h->device);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    Shape s{B, F, Hz, Wz, Lc, per_token, latent_dtype};
+    Shape s{B, F, Hz, Wz, Lc, per_token, latent_dtype, Li};
     Plan* plan = nullptr;
     wan_status ps = ensure_plan(h, s, &plan);
     if (ps != WAN_OK) return ps;
@@ -729,10 +814,11 @@ wan_status wan_dit_forward(wan_dit* h, const void* latent, int latent_dtype, int
     WAN_CU(cudaMemcpyAsync(h->lat_stage, latent, lat_bytes, h2d, st), "latent copy");
     WAN_CU(cudaMemcpyAsync(h->t_stage, timestep, (size_t)(per_token ? B * L : B) * 4, h2d, st), "timestep copy");
     WAN_CU(cudaMemcpyAsync(h->ctx_stage, context, (size_t)B * Lc * c.text_dim * 2, h2d, st), "context copy");
+    if (Li > 0) WAN_CU(cudaMemcpyAsync(h->img_stage, image, (size_t)B * Li * c.image_dim * 2, h2d, st), "image copy");
 
     const bool dump = h->dump != nullptr;
     const bool timed = h->timing;
-    if (timed) WAN_CU(plan->timer.ensure(16 * c.num_blocks + 64), "timing events");
+    if (timed) WAN_CU(plan->timer.ensure(20 * c.num_blocks + 64), "timing events");
     KTimer* tm = timed ? &plan->timer : nullptr;
     if (tm) tm->n = 0;
     if (h->use_graph && !dump) {
@@ -962,7 +1048,7 @@ wan_status wan_op_patchify(const void* latent, int latent_dtype, int B, int C, i
     if (B < 0 || C <= 0 || F <= 0 || Hz % 2 || Wz % 2 || Hz <= 0 || Wz <= 0) return WAN_ESHAPE;
     LaunchCtx ctx;
     if (!op_ctx(reinterpret_cast<cudaStream_t>(stream), &ctx)) return WAN_ECUDA;
-    return op_status(wan::launch_patchify(latent, latent_dtype, B, C, F, Hz, Wz, X, ctx));
+    return op_status(wan::launch_patchify(latent, latent_dtype, B, C, F, Hz, Wz, X, 4 * C, ctx));
 }
 
 wan_status wan_op_unpatchify(const float* rows, int B, int C, int F, int Hz, int Wz, float* velocity, void* stream) {
