@@ -166,10 +166,13 @@ def arm_config(workload, world):
     w = configs.workload(workload)
     cfg = w["cfg"]
     B, Cc, F, Hz, Wz = w["latent"]
-    return {"workload": workload, "model": "Wan2.1-T2V-1.3B shape" if "1.3b" in workload else cfg,
+    model = ("Wan2.1-T2V-1.3B shape" if "1.3b" in workload else
+             "Wan2.1-I2V-14B shape" if "i2v-14b" in workload else cfg)
+    extra = {"image_len": w["image_len"]} if w.get("image_len") else {}
+    return {**extra, "workload": workload, "model": model,
             "global_batch": world * B, "seq_len": F * (Hz // 2) * (Wz // 2), "text_len": w["text_len"],
             "blocks": cfg["num_blocks"], "timesteps": w["timesteps"], "parallelism": f"replicas x{world}",
-            "l2": "inputs larger than L2 (2.8 GB weights + GBs of activations per step); no flush"}
+            "l2": "inputs larger than L2 (GBs of weights and activations per step); no flush"}
 
 
 # ---------------------------------------------------------------- our arm
@@ -197,7 +200,9 @@ def run_ours(args, rank, world, local_rank):
         ts = [synth.make_timestep_per_token(B, L, (Hz // 2) * (Wz // 2), seed=args.seed).to(dev)]
     else:
         ts = [synth.make_timestep(B, v).to(dev) for v in w["timesteps"]]
-    dit = WanDiT(cfg, max_batch=B, max_tokens=L, max_text=Lc, device=local_rank)
+    Li = w.get("image_len", 0)   # image tokens per sample (I2V workloads)
+    img = synth.make_image(B, Li, cfg["image_dim"], seed=args.seed, device=str(dev)) if Li else None
+    dit = WanDiT(cfg, max_batch=B, max_tokens=L, max_text=Lc, device=local_rank, max_image=max(Li, 1))
     dit.load_weights(W)
     del W
     torch.cuda.synchronize()
@@ -205,7 +210,7 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
 
     def step(k):
-        dit.forward(lat, ts[k % len(ts)], ctx, velocity=vel)
+        dit.forward(lat, ts[k % len(ts)], ctx, velocity=vel, image=img)
 
     for k in range(args.warmup):
         step(k)
@@ -240,9 +245,10 @@ def run_ours(args, rank, world, local_rank):
     lat_h = lat.cpu().pin_memory()
     ctx_h = ctx.cpu().pin_memory()
     ts_h = [t.cpu().pin_memory() for t in ts]
+    img_h = img.cpu().pin_memory() if img is not None else None
     vel_h = torch.empty(vel.shape, dtype=torch.float32).pin_memory()
     for k in range(2):
-        dit.forward(lat_h, ts_h[k % len(ts_h)], ctx_h, velocity=vel_h)
+        dit.forward(lat_h, ts_h[k % len(ts_h)], ctx_h, velocity=vel_h, image=img_h)
     dit.sync()
     if world > 1:
         dist.barrier()
@@ -250,17 +256,17 @@ def run_ours(args, rank, world, local_rank):
     e2.record(stream)
     e2e_steps = max(1, min(args.steps, 3))
     for k in range(e2e_steps):
-        dit.forward(lat_h, ts_h[k % len(ts_h)], ctx_h, velocity=vel_h)
+        dit.forward(lat_h, ts_h[k % len(ts_h)], ctx_h, velocity=vel_h, image=img_h)
     e3.record(stream)
     dit.sync()
     ms_e2e = e2.elapsed_time(e3) / e2e_steps
     h2d = lat_h.numel() * lat_h.element_size() + ctx_h.numel() * ctx_h.element_size() + \
-        ts_h[0].numel() * ts_h[0].element_size()
+        ts_h[0].numel() * ts_h[0].element_size() + (img_h.numel() * img_h.element_size() if img_h is not None else 0)
     d2h = vel_h.numel() * vel_h.element_size()
 
     ms, ms_e2e = reduce_max([ms, ms_e2e], dev)
 
-    flops = dit.flops(B, F, Hz, Wz, Lc, int(w["timesteps"] == "per_token"))
+    flops = dit.flops(B, F, Hz, Wz, Lc, int(w["timesteps"] == "per_token"), Li)
     # dominant kernel: self-attention, 4 * L^2 * head_dim * heads * B flops per launch
     sa_ms, sa_n = kt["self_attention"]
     sa_flops = 4.0 * L * L * cfg["dim"] * B
@@ -291,8 +297,10 @@ def run_ours(args, rank, world, local_rank):
                      "peak": peak, "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None,
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
                      "flops_per_launch": sa_flops, "avg_launch_ms": sa_avg_ms, "launches_per_step": sa_n,
+                     # the committed ncu capture is of the default workload's self-attention launch
                      "traffic": measured_traffic("attn_tc_kernel",
-                                                 "video_diffusion_transformer_dit_b200/csrc/attention.cu"),
+                                                 "video_diffusion_transformer_dit_b200/csrc/attention.cu")
+                     if args.workload == DEFAULT_WORKLOAD else None,
                      "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
         "kernel_ms_per_step": {c: v[0] for c, v in kt.items()},
         "e2e": {"value": whole_job_tokens_per_s(world, B, L, ms_e2e), "unit": "tokens/s", "ms_per_step": ms_e2e,

@@ -41,6 +41,9 @@ WORKLOADS = {
     "wan-i2v-1blk-3x16x16": dict(model="wan2.1-i2v-14b",
                                  overrides=dict(dim=1536, heads=12, ffn_dim=8960, num_blocks=1),
                                  latent=(2, 36, 3, 16, 16), text_len=32, image_len=257, timesteps=(500.0,)),
+    # I2V route at Wan2.1-I2V-14B shapes, 81 frames 480x832 -> 32760 tokens, 257 image tokens
+    "wan-i2v-14b-81f-480x832": dict(model="wan2.1-i2v-14b", overrides={},
+                                    latent=(1, 36, 21, 60, 104), text_len=512, image_len=257, timesteps=(500.0,)),
     # Wan2.2-5B shape, 121 frames 704x1280 -> 27280 tokens, per-token timestep
     "wan5b-121f-704x1280-pertoken": dict(model="wan2.2-5b", overrides={},
                                          latent=(1, 48, 31, 44, 80), text_len=512, timesteps="per_token"),
