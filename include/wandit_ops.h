@@ -127,6 +127,24 @@ WANDIT_API wan_status wan_op_patchify(const void* latent, int latent_dtype, int 
 WANDIT_API wan_status wan_op_unpatchify(const float* rows, int B, int C, int F, int Hz, int Wz,
                              float* velocity, void* stream);
 
+/* Causal 3-D convolution of the Wan VAE decoder (pswp.cn WanPipeline notes,
+ * "WanCausalConv3d": 2 p_t zero frames before the input and none after, p_h /
+ * p_w zero rows / columns on both sides, p = (k - 1) / 2; with a cache of the
+ * frames right before frame 0 those replace the leading zero frames, as in the
+ * decoder's frame loop).  Channels-last bf16 tensors:
+ *   x      [B, T, H, W, Ci]            input frames (device)
+ *   cache  [B, nc, H, W, Ci] or NULL   the nc frames before frame 0 (nc <= kt - 1)
+ *   w      [Co, ldw] bf16: row co holds W[co, :, it, ih, iw] in (it, ih, iw, ci)
+ *          order, ci fastest, zero from kt*kh*kw*Ci up to ldw
+ *   bias   f32 [Co] or NULL;  y  [B, T, H, W, Co] output (device)
+ *   col    device workspace of at least B*T*H*W * ldw bf16 (the im2col rows)
+ * kt, kh, kw odd; Ci % 8 == 0; Co % 64 == 0; ldw = kt*kh*kw*Ci rounded up to a
+ * multiple of 64.  Runs as a gather into col plus the tcgen05 GEMM
+ * y = col . w^T + bias.  Returns WAN_ESHAPE for sizes outside these rules.  */
+WANDIT_API wan_status wan_op_causal_conv3d(const void* x, const void* cache, int nc, int B, int T, int H, int W,
+                                           int Ci, const void* w, int64_t ldw, const float* bias, int Co, int kt,
+                                           int kh, int kw, void* col, int64_t col_elems, void* y, void* stream);
+
 /* One flow-matching sampler step with classifier-free guidance
  * ("【VLA与模仿学习】Wan2.1框架与训练源码导读" §7: CFG  v = v_uncond + s (v_cond - v_uncond),
  * Euler update  x_next = x + (sigma_next - sigma) v; §6.1 x_sigma = (1 - sigma) z + sigma eps).

@@ -10,6 +10,7 @@ import pytest
 import torch
 
 from oracle import wan_oracle as O
+from oracle import wan_vae as V
 from tests.gpu_common import DT, bf16_round, need_gpu, rel_l2
 
 pytestmark = pytest.mark.gpu
@@ -286,3 +287,37 @@ def test_cfg_euler_matches_oracle_and_worked_example():
     B().op_cfg_euler(x1, vs, None, 1.0, 0.5, 0.0, x2)
     B().op_sync()
     assert torch.equal(x1.cpu(), torch.full((5,), 6.0)) and torch.equal(x2.cpu(), torch.full((5,), 2.0))
+
+
+# ------------------------------------------------------------------ VAE decoder: causal Conv3d
+
+@pytest.mark.parametrize("Ci,Co,kernel,T,nc", [(64, 128, (3, 3, 3), 3, 0), (16, 64, (3, 3, 3), 2, 2),
+                                               (64, 128, (3, 1, 1), 4, 1), (32, 64, (1, 1, 1), 2, 0)])
+def test_causal_conv3d_matches_oracle(Ci, Co, kernel, T, nc):
+    """Channels-last causal Conv3d (gather + tcgen05 GEMM) against the oracle's
+    WanCausalConv3d, with and without a cache of the frames before frame 0;
+    Ci = 16 exercises the zero-padded K (432 -> 448)."""
+    Bn, H, W = 2, 5, 7
+    kt, kh, kw = kernel
+    g = torch.Generator().manual_seed(Ci + Co + T + nc)
+    x = torch.randn(Bn, Ci, T, H, W, generator=g).to(torch.bfloat16)
+    w = (torch.randn(Co, Ci, kt, kh, kw, generator=g) * 0.05).to(torch.bfloat16)
+    bias = torch.randn(Co, generator=g) * 0.1
+    cache = torch.randn(Bn, Ci, nc, H, W, generator=g).to(torch.bfloat16) if nc else None
+    ref = V.causal_conv3d(x.to(DT), w.to(DT), bias.to(DT), cache.to(DT) if nc else None)
+    K = kt * kh * kw * Ci
+    Kp = (K + 63) // 64 * 64
+    wp = torch.zeros(Co, Kp, dtype=torch.bfloat16)
+    wp[:, :K] = w.permute(0, 2, 3, 4, 1).reshape(Co, K)
+    xd = x.permute(0, 2, 3, 4, 1).contiguous().cuda()
+    cd = cache.permute(0, 2, 3, 4, 1).contiguous().cuda() if nc else None
+    col = torch.empty(Bn * T * H * W * Kp, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(Bn, T, H, W, Co, dtype=torch.bfloat16, device="cuda")
+    B_ = B()
+    B_.op_causal_conv3d(xd, wp.cuda(), bias.cuda(), col, y, kernel, cache=cd)
+    B_.op_sync()
+    got = y.cpu().permute(0, 4, 1, 2, 3)
+    assert rel_l2(got, ref) < TOL
+    with pytest.raises(B_.WanError):                 # Co must be a multiple of 64
+        B_.op_causal_conv3d(xd, wp[:32].contiguous().cuda(), None, col, y[..., :32].contiguous(), kernel, cache=cd)
+

@@ -31,7 +31,7 @@ SYMBOLS = ["wan_dit_create", "wan_dit_load_weights", "wan_dit_missing_weights", 
            "wan_dit_last_error", "wan_status_string", "wan_dit_destroy",
            "wan_op_gemm", "wan_op_attention", "wan_op_layernorm", "wan_op_rmsnorm_rope", "wan_op_patchify",
            "wan_op_unpatchify", "wan_op_sync", "wan_op_set_wait_limit_ns", "wan_op_rmsnorm_rope_noalloc", "wan_op_cfg_euler",
-           "wan_op_wait_selftest"]
+           "wan_op_wait_selftest", "wan_op_causal_conv3d"]
 
 
 class WanError(RuntimeError):
@@ -96,6 +96,7 @@ def lib() -> C.CDLL:
         "wan_op_sync": (I, [P]),
         "wan_op_cfg_euler": (I, [P, P, P, F, F, F, I64, P, P]),
         "wan_op_wait_selftest": (I, [I64, P]),
+        "wan_op_causal_conv3d": (I, [P, P, I, I, I, I, I, I, P, I64, P, I, I, I, I, P, I64, P, P]),
         "wan_op_set_wait_limit_ns": (None, [I64]),
     }
     for name, (res, args) in sig.items():
@@ -284,6 +285,19 @@ def op_gemm(A, W, epilogue: str, out, bias=None, gate0=None, gate1=None, mod_div
                      up_C=unpatch[0], up_F=unpatch[1], up_Hz=unpatch[2], up_Wz=unpatch[3])
     _check(lib().wan_op_gemm(_ptr(A), A.stride(0), _ptr(W), W.stride(0), M, N, K, EPI[epilogue], C.byref(e),
                              _stream(stream)), "wan_op_gemm")
+
+
+def op_causal_conv3d(x, w_packed, bias, col, y, kernel, cache=None, stream=None):
+    """x bf16 [B,T,H,W,Ci], w_packed bf16 [Co, ldw] ((kt,kh,kw,ci) order, zero padded
+    to ldw), bias f32 [Co] or None, col bf16 workspace, y bf16 [B,T,H,W,Co],
+    kernel (kt, kh, kw), cache bf16 [B,nc,H,W,Ci] or None (channels last)."""
+    B, T, H, W, Ci = x.shape
+    Co = w_packed.shape[0]
+    kt, kh, kw = kernel
+    nc = 0 if cache is None else cache.shape[1]
+    _check(lib().wan_op_causal_conv3d(_ptr(x), _ptr(cache), nc, B, T, H, W, Ci, _ptr(w_packed), w_packed.stride(0),
+                                      _ptr(bias), Co, kt, kh, kw, _ptr(col), col.numel(), _ptr(y), _stream(stream)),
+           "wan_op_causal_conv3d")
 
 
 def op_attention(q, k, v, o, B, heads, Lq, Lk, ldq=None, ldk=None, ldv=None, ldo=None, stream=None):

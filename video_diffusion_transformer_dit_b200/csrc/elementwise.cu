@@ -388,6 +388,58 @@ cudaError_t launch_patchify(const void* latent, int latent_dtype, int B, int C, 
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ causal Conv3d im2col (channels last)
+// col[row, k] for row = ((b * T + t) * H + h) * W + w and k = tap * Ci + c,
+// tap = (it * kh + ih) * kw + iw: the input at frame t - (kt - 1) + it,
+// row h - (kh - 1) / 2 + ih, column w - (kw - 1) / 2 + iw, channel c.  Frames
+// before 0 come from the cache (its last frames sit right before frame 0),
+// else zero; rows/columns outside the frame are zero; k in [taps * Ci, Kp) is
+// zero padding.  8 channels (16 bytes) per thread step.
+__global__ void causal_im2col_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ cache,
+                                     int nc, int B, int T, int H, int W, int Ci, int kt, int kh, int kw,
+                                     __nv_bfloat16* __restrict__ col, int Kp) {
+    const int C8 = Ci >> 3, Kp8 = Kp >> 3;
+    const long long K8 = (long long)kt * kh * kw * C8;
+    const long long total = (long long)B * T * H * W * Kp8;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const long long row = idx / Kp8;
+        const int k8 = (int)(idx - row * Kp8);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (k8 < K8) {
+            const int tap = k8 / C8, c8 = k8 - tap * C8;
+            const int it = tap / (kh * kw), ih = (tap / kw) % kh, iw = tap % kw;
+            const int w0 = (int)(row % W);
+            const int h0 = (int)((row / W) % H);
+            const int t0 = (int)((row / ((long long)W * H)) % T);
+            const int b0 = (int)(row / ((long long)W * H * T));
+            const int tt = t0 - (kt - 1) + it, hh = h0 - (kh - 1) / 2 + ih, ww = w0 - (kw - 1) / 2 + iw;
+            if (hh >= 0 && hh < H && ww >= 0 && ww < W) {
+                if (tt >= 0)
+                    v = *reinterpret_cast<const uint4*>(x + ((((long long)b0 * T + tt) * H + hh) * W + ww) * Ci + c8 * 8);
+                else if (cache && tt >= -nc)
+                    v = *reinterpret_cast<const uint4*>(
+                        cache + ((((long long)b0 * nc + (nc + tt)) * H + hh) * W + ww) * Ci + c8 * 8);
+            }
+        }
+        *reinterpret_cast<uint4*>(col + row * Kp + (long long)k8 * 8) = v;
+    }
+}
+
+cudaError_t launch_causal_im2col(const void* x, const void* cache, int nc, int B, int T, int H, int W, int Ci, int kt,
+                                 int kh, int kw, void* col, int Kp, const LaunchCtx& ctx) {
+    if (Ci % 8 || Kp % 8 || (long long)kt * kh * kw * Ci > Kp) return cudaErrorInvalidValue;
+    const long long total = (long long)B * T * H * W * (Kp / 8);
+    if (total <= 0) return cudaSuccess;
+    long long g = (total + 255) / 256;
+    if (g > ctx.num_sms * 16) g = ctx.num_sms * 16;
+    causal_im2col_kernel<<<(int)g, 256, 0, ctx.stream>>>(reinterpret_cast<const __nv_bfloat16*>(x),
+                                                        reinterpret_cast<const __nv_bfloat16*>(cache), nc, B, T, H, W,
+                                                        Ci, kt, kh, kw, reinterpret_cast<__nv_bfloat16*>(col), Kp);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ a += b (bf16, fp32 sum, one rounding)
 __global__ void add_bf16_kernel(__nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b, long long n8) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {

@@ -85,6 +85,10 @@ cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float 
 
 cudaError_t launch_patchify(const void* latent, int latent_dtype, int B, int C, int F, int Hz, int Wz, void* X,
                             int ldx, const LaunchCtx& ctx);  // ldx >= 4C: row stride of X, pad columns zeroed
+// Causal Conv3d im2col, channels last: col [B*T*H*W, Kp] bf16 (Kp >= kt*kh*kw*Ci, pad zeroed),
+// cache [B, nc, H, W, Ci] (frames right before frame 0) or null.
+cudaError_t launch_causal_im2col(const void* x, const void* cache, int nc, int B, int T, int H, int W, int Ci, int kt,
+                                 int kh, int kw, void* col, int Kp, const LaunchCtx& ctx);
 // a[i] = bf16(a[i] + b[i]) for n bf16 values (n % 8 == 0, 16-byte aligned)
 cudaError_t launch_add_bf16(void* a, const void* b, long long n, const LaunchCtx& ctx);
 cudaError_t launch_unpatchify(const float* rows, int B, int C, int F, int Hz, int Wz, float* vel,

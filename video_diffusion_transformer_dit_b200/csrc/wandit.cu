@@ -1051,6 +1051,33 @@ wan_status wan_op_patchify(const void* latent, int latent_dtype, int B, int C, i
     return op_status(wan::launch_patchify(latent, latent_dtype, B, C, F, Hz, Wz, X, 4 * C, ctx));
 }
 
+wan_status wan_op_causal_conv3d(const void* x, const void* cache, int nc, int B, int T, int H, int W, int Ci,
+                                const void* w, int64_t ldw, const float* bias, int Co, int kt, int kh, int kw, void* col,
+                                int64_t col_elems, void* y, void* stream) {
+    if (!x || !w || !col || !y) return WAN_EINVAL;
+    if (B <= 0 || T <= 0 || H <= 0 || W <= 0 || Ci <= 0 || Co <= 0) return WAN_ESHAPE;
+    if (kt <= 0 || kh <= 0 || kw <= 0 || !(kt & 1) || !(kh & 1) || !(kw & 1)) return WAN_ESHAPE;
+    if (Ci % 8 || Co % 64 || nc < 0 || nc > kt - 1 || (nc > 0 && !cache)) return WAN_ESHAPE;
+    const long long K = (long long)kt * kh * kw * Ci, Kp = (K + 63) / 64 * 64;
+    if (ldw != Kp || Kp > (1LL << 30)) return WAN_ESHAPE;
+    const long long M = (long long)B * T * H * W;
+    if (M > (1LL << 31) - 1 || col_elems < M * Kp) return WAN_ESHAPE;
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(col) | reinterpret_cast<uintptr_t>(w) |
+         reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(cache)) & 15)
+        return WAN_EINVAL;
+    LaunchCtx ctx;
+    if (!op_ctx(reinterpret_cast<cudaStream_t>(stream), &ctx)) return WAN_ECUDA;
+    cudaError_t e = wan::launch_causal_im2col(x, nc > 0 ? cache : nullptr, nc, B, T, H, W, Ci, kt, kh, kw, col, (int)Kp, ctx);
+    if (e != cudaSuccess) return op_status(e);
+    EpiParams p{};
+    p.kind = wan::EPI_BIAS;
+    p.bias = bias;
+    p.out = y;
+    p.ldo = Co;
+    p.mod_div = 1;
+    return op_status(wan::launch_gemm(col, Kp, w, Kp, (int)M, Co, (int)Kp, p, ctx));
+}
+
 wan_status wan_op_unpatchify(const float* rows, int B, int C, int F, int Hz, int Wz, float* velocity, void* stream) {
     if (!rows || !velocity) return WAN_EINVAL;
     if (B < 0 || C <= 0 || F <= 0 || Hz % 2 || Wz % 2 || Hz <= 0 || Wz <= 0) return WAN_ESHAPE;
