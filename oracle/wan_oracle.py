@@ -55,6 +55,12 @@ R20 I2V image cross-attention: the image tokens (placed before the text tokens
 R21 MoE expert switch: with t decreasing over sampling, steps with
     t >= boundary * num_train_timesteps use the high-noise expert and the rest
     the low-noise expert; both forwards of a CFG step use the same expert.
+R22 flow shift: the pages give only the value (3.0 at 480p, 5.0 at 720p) and
+    where it acts (the scheduler's timestep set-up); taken as the usual
+    flow-matching time shift sigma' = s sigma / (1 + (s - 1) sigma), which
+    multiplies the noise odds sigma / (1 - sigma) by s, applied to the uniform
+    ladder sigma_i = 1 - i / steps (i = 0 .. steps - 1) with a final 0, and
+    timesteps t_i = sigma_i * num_train_timesteps.
 
 Parity unpinned (conventions the pages do not fix, so no pin can tell a
 right reading from a wrong one; the oracle and the CUDA path simply agree):
@@ -567,3 +573,29 @@ def moe_expert(t: float, boundary: float, num_train_timesteps: int = 1000) -> in
 def euler_step(x, sigma, sigma_next, v):
     """x_next = x + (sigma_next - sigma) v ([WAN21-GUIDE] §7)."""
     return x + (sigma_next - sigma) * v
+
+
+def flow_shift(sigma, shift: float):
+    """Shifted noise level s sigma / (1 + (s - 1) sigma) (reading R22).  The
+    shift value is set per resolution in the pipeline set-up of [PSWP-WAN]
+    (flow_shift 3.0 at 480p, 5.0 at 720p) and takes effect where the scheduler
+    builds its timesteps ([WAN22-PITFALLS] "shift 参数生效了两次,在两个地方")."""
+    sigma = torch.as_tensor(sigma, dtype=DT)
+    return shift * sigma / (1.0 + (shift - 1.0) * sigma)
+
+
+def sampling_sigmas(steps: int, shift: float) -> torch.Tensor:
+    """Noise levels of a `steps`-step sampling run, steps + 1 values from 1 down
+    to a final 0: the uniform ladder 1 - i / steps (i < steps) shifted by
+    flow_shift, then 0 for the last Euler update to land on (R22; the Euler
+    update of [WAN21-GUIDE] §7 walks sigma to sigma_next)."""
+    if steps < 1:
+        raise ValueError("steps must be >= 1")
+    ladder = 1.0 - torch.arange(steps, dtype=DT) / steps
+    return torch.cat([flow_shift(ladder, shift), torch.zeros(1, dtype=DT)])
+
+
+def sampling_timesteps(steps: int, shift: float, num_train_timesteps: int = 1000) -> torch.Tensor:
+    """Timestep values the DiT (and the expert switch) sees: sigma * num_train_timesteps
+    for the first `steps` noise levels (R22)."""
+    return sampling_sigmas(steps, shift)[:steps] * num_train_timesteps

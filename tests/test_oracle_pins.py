@@ -665,3 +665,97 @@ def test_cfg_combine_endpoints():
     assert torch.equal(O.cfg_combine(vu, vc, 0.0), vu)
     torch.testing.assert_close(O.cfg_combine(vu, vc, 1.0), vc, rtol=0, atol=1e-15)
     torch.testing.assert_close(O.cfg_combine(vu, vc, 6.0), vu + 6.0 * (vc - vu))
+
+
+# ---------------------------------------------------------------- conditioning MLPs against library layers
+
+def test_text_embedding_is_two_linears_around_gelu():
+    """R4 (config of the smallest case: Linear-GELU-Linear, GELU in its tanh
+    form): the text path against torch's own linear and tanh-GELU layers."""
+    cfg = tiny_cfg()
+    W = rand_weights(cfg, seed=21)
+    ctx = torch.randn(2, 5, cfg["text_dim"], generator=torch.Generator().manual_seed(22), dtype=DT)
+    p = "condition_embedder.text_embedder."
+    h = Fn.linear(ctx, W[p + "linear_1.weight"], W[p + "linear_1.bias"])
+    ref = Fn.linear(Fn.gelu(h, approximate="tanh"), W[p + "linear_2.weight"], W[p + "linear_2.bias"])
+    torch.testing.assert_close(O.text_embedding(ctx, W), ref, rtol=1e-12, atol=1e-13)
+    # the activation matters at this scale: a dropped or exact-erf GELU would not match
+    assert (Fn.linear(h, W[p + "linear_2.weight"], W[p + "linear_2.bias"]) - ref).abs().max() > 1e-3
+    erf = Fn.linear(Fn.gelu(h), W[p + "linear_2.weight"], W[p + "linear_2.bias"])
+    assert (erf - ref).abs().max() > 1e-6
+
+
+def test_time_embedding_wiring():
+    """R3: temb = L2(SiLU(L1(sinusoid(t)))), timestep_proj = Lp(SiLU(temb)) of
+    width 6D, unflattened to [6, D] chunk by chunk -- against torch's linear and
+    SiLU layers; the printed shapes temb (1, D), projection (1, 6D) -> (1, 6, D)
+    are those of the 480p listing."""
+    cfg = tiny_cfg()
+    W = rand_weights(cfg, seed=23)
+    D = cfg["dim"]
+    t = torch.tensor([999.0, 500.0, 20.0], dtype=DT)
+    p = "condition_embedder."
+    e = O.timestep_sinusoid(t, cfg["freq_dim"])
+    h = Fn.silu(Fn.linear(e, W[p + "time_embedder.linear_1.weight"], W[p + "time_embedder.linear_1.bias"]))
+    temb_ref = Fn.linear(h, W[p + "time_embedder.linear_2.weight"], W[p + "time_embedder.linear_2.bias"])
+    proj_ref = Fn.linear(Fn.silu(temb_ref), W[p + "time_proj.weight"], W[p + "time_proj.bias"])
+    temb, proj = O.time_embedding(t, W, cfg)
+    assert temb.shape == (3, D) and proj.shape == (3, 6, D)
+    torch.testing.assert_close(temb, temb_ref, rtol=1e-12, atol=1e-13)
+    for k in range(6):      # chunk k of the 6D projection is modulation row k
+        torch.testing.assert_close(proj[:, k], proj_ref[:, k * D:(k + 1) * D], rtol=1e-12, atol=1e-13)
+    # per-token timesteps [B, L] give per-token rows of the same map
+    tt = torch.tensor([[0.0, 250.0], [999.0, 20.0]], dtype=DT)
+    temb2, proj2 = O.time_embedding(tt, W, cfg)
+    assert temb2.shape == (2, 2, D) and proj2.shape == (2, 2, 6, D)
+    torch.testing.assert_close(temb2[1, 0], O.time_embedding(tt[1, :1], W, cfg)[0][0], rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- flow-shift schedule (reading R22)
+
+def test_flow_shift_values_and_closed_forms():
+    g = GOLD["flow_shift"]
+    assert g["480p"] == 3.0 and g["720p"] == 5.0
+    sig = torch.linspace(0, 1, 101, dtype=DT)
+    for s in (g["480p"], g["720p"], 0.5, 1.7):
+        y = O.flow_shift(sig, s)
+        assert y[0].item() == 0.0 and y[-1].item() == 1.0              # endpoints stay
+        assert bool((y[1:] > y[:-1]).all())                             # order of noise levels kept
+        mid = sig[1:-1]
+        ym = y[1:-1]
+        torch.testing.assert_close(ym / (1 - ym), s * mid / (1 - mid), rtol=1e-12, atol=0)  # odds times s
+        if s > 1:
+            assert bool((ym > mid).all())                               # more of the run at high noise
+    # the shift is a one-parameter group: applied twice it compounds (the pitfall the
+    # pages warn of), the constructor's fixed 1 is neutral, and 1/s undoes s
+    for a, b in ((3.0, 5.0), (2.0, 0.25)):
+        torch.testing.assert_close(O.flow_shift(O.flow_shift(sig, a), b), O.flow_shift(sig, a * b),
+                                   rtol=1e-12, atol=1e-15)
+    torch.testing.assert_close(O.flow_shift(O.flow_shift(sig, g["constructor_shift"]), 3.0), O.flow_shift(sig, 3.0),
+                               rtol=0, atol=1e-16)
+    torch.testing.assert_close(O.flow_shift(O.flow_shift(sig, 5.0), 1 / 5.0), sig, rtol=1e-12, atol=1e-15)
+    assert abs(O.flow_shift(0.5, 3.0).item() - 0.75) < 1e-15            # s / (1 + s) at the midpoint
+
+
+def test_sampling_sigmas_and_timesteps():
+    for steps in (1, 4, 50):
+        torch.testing.assert_close(O.sampling_sigmas(steps, 1.0),
+                                   torch.linspace(1, 0, steps + 1, dtype=DT), rtol=0, atol=1e-15)
+    s = O.sampling_sigmas(50, 3.0)
+    assert s.shape == (51,) and s[0].item() == 1.0 and s[-1].item() == 0.0
+    assert bool((s[1:] < s[:-1]).all())
+    ts = O.sampling_timesteps(50, 3.0)
+    assert ts.shape == (50,) and ts[0].item() == 1000.0
+    torch.testing.assert_close(ts, s[:50] * 1000)
+    # the Euler walk over the schedule with the exact velocity lands on the data
+    # (the worked example's straight path, at every step count and shift)
+    z, eps = torch.tensor(2.0, dtype=DT), torch.tensor(10.0, dtype=DT)
+    for steps, shift in ((4, 1.0), (7, 3.0), (30, 5.0)):
+        sig = O.sampling_sigmas(steps, shift)
+        x = O.flow_interpolate(z, eps, sig[0])
+        for i in range(steps):
+            x = O.euler_step(x, sig[i], sig[i + 1], O.flow_target(z, eps))
+        assert abs(x.item() - 2.0) < 1e-12
+    # a larger shift keeps more steps above the A14B switch point (the drift the pages warn of)
+    hi = [int((O.sampling_timesteps(50, s) >= 875.0).sum()) for s in (1.0, 3.0, 5.0)]
+    assert hi[0] < hi[1] < hi[2]
