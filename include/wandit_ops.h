@@ -25,9 +25,10 @@ extern "C" {
  *  WAN_EPI_BIAS          out bf16 = acc + bias[c]                       (every nn.Linear)
  *  WAN_EPI_BIAS_GELU     out bf16 = GELU_tanh(acc + bias[c])            (ffn.net.0 + activation;
  *                        text_embedder linear_1 + activation)
- *  WAN_EPI_GATE_RESIDUAL out bf16 = out + (acc + bias[c]) * gate(r, c)  ("hidden_states.float()
- *                        + attn_output * gate_msa" / "+ ff_output * c_gate_msa" in
- *                        WanTransformerBlock), gate(r, c) = gate0[c] + gate1[(r / mod_div) * mod_ld + c]
+ *  WAN_EPI_GATE_RESIDUAL out bf16 = out + (acc + bias[c]) * gate(r, c)  (the gated residual
+ *                        x + gate_msa * attn1(..) and x + c_gate_msa * ffn(..) of the pswp.cn
+ *                        notes, section "WanTransformerBlock", added in fp32),
+ *                        gate(r, c) = gate0[c] + gate1[(r / mod_div) * mod_ld + c]
  *  WAN_EPI_RESIDUAL      out bf16 = out + bf16(acc + bias[c])           (cross-attention residual)
  *  WAN_EPI_BIAS_F32      out f32  = acc + bias[c]
  *  WAN_EPI_UNPATCHIFY    velocity f32 = bf16(acc + bias[c]) scattered by the unpatchify map
@@ -102,8 +103,11 @@ WANDIT_API wan_status wan_op_rmsnorm_rope(void* buf, int64_t ld, int rows, int D
  * loading the library holds until the process exits, and calls no cudaMalloc,
  * cudaFree or other allocating routine.
  *  - Limit: Fp, Hp and Wp (post-patch grid) must each be <= 1024, the
- *    rope_max_seq_len of the Wan configs; larger grids return WAN_ESHAPE
- *    before anything is launched.
+ *    rope_max_seq_len of the Wan configs; larger grids, and D / ld outside
+ *    the rules of wan_op_rmsnorm_rope, return WAN_ESHAPE before the array is
+ *    touched or anything is launched.  A CUDA error already pending on the
+ *    calling thread is returned as WAN_ECUDA, also before any launch (and
+ *    left pending for the caller).
  *  - The first call on a device (with that device current) looks up the
  *    array's device address with cudaGetSymbolAddress and caches it; make
  *    that first call before any stream capture on the device.

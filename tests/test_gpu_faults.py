@@ -42,16 +42,19 @@ def test_forward_with_zero_wait_limit_reports_and_recovers():
     L, Lc = O.token_count(*lat.shape[2:]), ctx.shape[1]
     dit = make_dit(cfg, 1, L, Lc, W)
     ref = dit.forward(lat.cuda(), t.cuda(), ctx.cuda(), sync=True).cpu()
+    # a limit of 0 gives up at the first probe that finds a barrier still open;
+    # every forward has such waits (each TMA load takes time to land)
     dit.set_option(WAN_OPT_WAIT_LIMIT_NS, 0)
-    status = "WAN_OK"
+    seen = []
     for _ in range(3):
         dit.forward(lat.cuda(), t.cuda(), ctx.cuda())
         try:
             dit.sync()
+            seen.append("WAN_OK")
         except WanError as e:
-            status = e.name
-            break
-    assert status in ("WAN_ETIMEOUT", "WAN_OK")
+            seen.append(e.name)
+    assert "WAN_ETIMEOUT" in seen, seen
+    assert set(seen) <= {"WAN_ETIMEOUT", "WAN_OK"}, seen
     dit.set_option(WAN_OPT_WAIT_LIMIT_NS, 2_000_000_000)
     again = dit.forward(lat.cuda(), t.cuda(), ctx.cuda(), sync=True).cpu()
     assert torch.equal(again, ref)

@@ -5,8 +5,9 @@ while they run (their own pool allocator owns HBM, or they cannot take the
 synchronisation an allocation may cause).  It keeps its cos/sin table in a
 fixed device array; this test calls it through the C ABI twice in a row, on
 two different grids, and checks each result against wan_op_rmsnorm_rope on
-the same input with the tolerance of the other kernel tests, then checks that
-a grid beyond the array's 1024 positions per axis is refused.  The file name
+the same input with the tolerance of the other kernel tests, checks one grid
+against the float64 oracle directly, then checks that bad widths and strides
+and a grid beyond the array's 1024 positions per axis are refused.  The file name
 makes pytest collect it last.
 """
 import pytest
@@ -45,6 +46,32 @@ def test_noalloc_matches_allocating_op_twice(B):
         err = _rel_l2(got[:, D:2 * D], ref[:, D:2 * D])
         assert err < TOL, f"call {call}: rel-L2 {err}"
         assert torch.equal(got[:, :D].cpu(), x[:, :D]) and torch.equal(got[:, 2 * D:].cpu(), x[:, 2 * D:])
+
+
+def test_noalloc_matches_oracle(B):
+    """The fixed-array table path against the float64 oracle's RMSNorm across
+    heads and 3-axis rotation directly (not only against the other CUDA op)."""
+    from oracle import wan_oracle as O
+    Fp, Hp, Wp = 3, 5, 7
+    L, D = Fp * Hp * Wp, 1536
+    x = torch.randn(2 * L, D, generator=torch.Generator().manual_seed(30)).to(torch.bfloat16)
+    gain = 1 + 0.1 * torch.randn(D, generator=torch.Generator().manual_seed(31))
+    got = x.cuda()
+    B.op_rmsnorm_rope_noalloc(got.data_ptr(), D, 2 * L, D, 1e-6, gain.cuda(), rope=True, grid=(Fp, Hp, Wp))
+    torch.cuda.synchronize()
+    ref = O.rms_norm(x.double(), 1e-6, gain.double())
+    ref = O.rope_apply(ref.reshape(2, L, 12, 128), O.rope_angles((Fp, Hp, Wp), (44, 42, 42), 10000.0))
+    assert _rel_l2(got, ref.reshape(2 * L, D)) < TOL
+
+
+def test_noalloc_rejects_bad_shapes_before_launch(B):
+    D = 1536
+    buf = torch.zeros(4, D, dtype=torch.bfloat16, device="cuda")
+    gain = torch.ones(D, device="cuda")
+    for args in ((D + 8, D), (D, D + 4), (D, D // 2)):       # width not a kernel width, odd stride, stride < D
+        with pytest.raises(B.WanError) as e:
+            B.op_rmsnorm_rope_noalloc(buf.data_ptr(), args[1], 4, args[0], 1e-6, gain, rope=True, grid=(1, 2, 2))
+        assert e.value.name == "WAN_ESHAPE"
 
 
 def test_noalloc_rejects_grid_beyond_table(B):

@@ -42,10 +42,7 @@ struct AttnParams {
 namespace attn {
 constexpr int TILE_BYTES = 128 * 128 * 2;  // one 128 x 128 bf16 tile = two 64-column swizzled halves
 constexpr int HALF_BYTES = 128 * 128;      // 128 rows x 128 bytes
-#ifndef WAN_ATTN_KSTAGES
-#define WAN_ATTN_KSTAGES 2
-#endif
-constexpr int KSTAGES = WAN_ATTN_KSTAGES;
+constexpr int KSTAGES = 2;                         // K ring slots (a third measured neutral)
 constexpr int VSTAGES = 2;
 constexpr int SQ = 0;                              // Q0 | Q1
 constexpr int SK = SQ + 2 * TILE_BYTES;            // K ring
@@ -54,34 +51,14 @@ constexpr int SBAR = SV + VSTAGES * TILE_BYTES;
 constexpr int SMEM_BYTES = SBAR + 256 + 1024;
 constexpr int THREADS = 384;
 constexpr int REGS_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
-#ifndef WAN_ATTN_REGS_CONTROL
-#define WAN_ATTN_REGS_CONTROL 88
-#define WAN_ATTN_REGS_SOFTMAX 208
-#endif
-constexpr int REGS_CONTROL = WAN_ATTN_REGS_CONTROL;  // warpgroup 0: producer + MMA issuer
-constexpr int REGS_SOFTMAX = WAN_ATTN_REGS_SOFTMAX;  // warpgroups 1, 2
+constexpr int REGS_CONTROL = 88;   // warpgroup 0: producer + MMA issuer
+constexpr int REGS_SOFTMAX = 208;  // warpgroups 1, 2
 static_assert(128 * REGS_CONTROL + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH, "register split");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
-// Column pairs per 8 whose exp2 runs as the FMA-pipe cubic instead of on the
-// MUFU.  0 by default: scalar FP32 work in the softmax warps competes with the
-// MMA-issuing warp on the same sub-partitions (measured: a tight tcgen05.mma
-// issue loop drops to a third of the tensor rate next to FFMA-bound warps, and
-// is unaffected by MUFU-, integer- or packed-f32x2-bound ones), which costs
-// more than the MUFU time the emulation saves.
-#ifndef WAN_ATTN_EMU_PAIRS
-#define WAN_ATTN_EMU_PAIRS 0
-#endif
-#ifndef WAN_ATTN_EX2_F32
-#define WAN_ATTN_EX2_F32 1   // 1: one ex2.approx.f32 per exponential; 0: ex2.approx.f16x2 pairs (measured slower)
-#endif
-constexpr int EMU_PAIRS_OF_8 = WAN_ATTN_EMU_PAIRS;  // column pairs per 8 on the software exp2
-#ifndef WAN_ATTN_PV_PARTS
-#define WAN_ATTN_PV_PARTS 2
-#endif
-// P.V issued in 2 or 4 parts over the 128 keys of a tile (measured at the 480p
-// shape: 2 parts ~1210 TFLOP/s, 4 parts ~1035, one part ~1060 with this issuer)
-constexpr int PV_PARTS = WAN_ATTN_PV_PARTS;
-static_assert(PV_PARTS == 2 || PV_PARTS == 4, "PV_PARTS");
+// P.V of a key tile goes in two K = 64 halves, the first issued as soon as the
+// softmax has stored the probabilities of keys 0..63 (measured at the 480p
+// shape: two parts ~1210 TFLOP/s, four ~1035, one ~1060).
+constexpr int PV_PARTS = 2;
 }  // namespace attn
 
 __global__ void __launch_bounds__(attn::THREADS, 1)
@@ -141,13 +118,16 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // producer: ring slots with a load issued and the phase it completes; MMA
+    // issuer: whether any MMA went out (both drained after an abort, before exit)
+    uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
+    bool issued = false;
 
     if (warp < 4) {
         regs_dealloc<REGS_CONTROL>();
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- producer ----------------
-            uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
             bool ok = true;
             mbar_expect_tx(q_full, 2 * TILE_BYTES);
             for (int t = 0; t < 2; ++t) {
@@ -170,13 +150,6 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                 varmed |= 1u << vs;
                 vpar = (vpar & ~(1u << vs)) | (vp << vs);
             }
-            if (!ok) {  // drain the loads still in flight before the CTA exits
-                mbar_drain(q_full, 0, 200000000ull);
-                for (int s = 0; s < KSTAGES; ++s)
-                    if (karmed & (1u << s)) mbar_drain(k_full + s, (kpar >> s) & 1, 200000000ull);
-                for (int s = 0; s < VSTAGES; ++s)
-                    if (varmed & (1u << s)) mbar_drain(v_full + s, (vpar >> s) & 1, 200000000ull);
-            }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -197,7 +170,6 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             return __shfl_sync(0xffffffffu, r, 0) != 0;
         };
         bool ok = wait(q_full, 0);
-        bool issued = false;
         // S_t(j) = Q_t K_j^T into TMEM columns [128 t, 128 t + 128)
         auto issue_s = [&](int t, int j) -> bool {
             const int ks = j % KSTAGES;
@@ -257,11 +229,6 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             if (!issue_pv_all(1, j)) { ok = false; break; }
             if (j + 1 < nk && !issue_s(1, j + 1)) { ok = false; break; }
         }
-        if (!ok && issued && elect_one()) {  // let the tensor core finish before TMEM is freed
-            umma_commit(drain);
-            mbar_drain(drain, 0, 200000000ull);
-        }
-        __syncwarp();
     }
     } else {
         regs_alloc<REGS_SOFTMAX>();
@@ -321,9 +288,10 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     tmem_st32(TO + c * 32, ov);
                 }
             }
-            // probabilities on packed fp32 pairs (EMU_PAIRS_OF_8 of every 8 pairs on the
-            // software exp2); each 32-column chunk is packed to bf16 and
-            // stored over its own S columns (P_t = first 64 columns of S_t) at once
+            // probabilities on packed fp32 pairs, every exponential on the MUFU (scalar
+            // FP32 work here would slow the MMA issue on the same sub-partitions);
+            // each 32-column chunk is packed to bf16 and stored over its own S
+            // columns (P_t = first 64 columns of S_t) at once
             uint64_t ps2[2] = {0ull, 0ull};
             const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
             const uint64_t negm2 = f2pack(-m_use, -m_use);
@@ -333,19 +301,9 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     const uint64_t x2 = fma2(f2pack(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])), scale2, negm2);
-                    float e0, e1;
-                    if (((i >> 1) & 7) >= 8 - EMU_PAIRS_OF_8) {
-                        ex2_poly2(x2, e0, e1);
-                    } else {
-                        float x0, x1;
-                        f2unpack(x2, x0, x1);
-#if WAN_ATTN_EX2_F32
-                        e0 = ex2_approx(x0);
-                        e1 = ex2_approx(x1);
-#else
-                        ex2_f16x2(x0, x1, e0, e1);
-#endif
-                    }
+                    float x0, x1;
+                    f2unpack(x2, x0, x1);
+                    const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
                     ps2[(i >> 1) & 1] = add2(ps2[(i >> 1) & 1], f2pack(e0, e1));
                     pc[i / 2] = pack_bf16(e0, e1);
                 }
@@ -396,6 +354,23 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // a wait gave up somewhere in the CTA: let this CTA's own loads and MMAs
+        // land (bounded) before its shared and tensor memory are released
+        if (warp == 0 && lane == 0) {
+            mbar_drain(q_full, 0, 200000000ull);
+            for (int s = 0; s < KSTAGES; ++s)
+                if (karmed & (1u << s)) mbar_drain(k_full + s, (kpar >> s) & 1, 200000000ull);
+            for (int s = 0; s < VSTAGES; ++s)
+                if (varmed & (1u << s)) mbar_drain(v_full + s, (vpar >> s) & 1, 200000000ull);
+        } else if (warp == 1 && issued) {
+            if (elect_one()) {  // the lane that issued the MMAs
+                umma_commit(drain);
+                mbar_drain(drain, 0, 200000000ull);
+            }
+            __syncwarp();
+        }
+    }
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();

@@ -53,19 +53,12 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                  : "memory");
 }
 
-#ifndef WAN_MBAR_TEST_WAIT
-#define WAN_MBAR_TEST_WAIT 1
-#endif
 // Non-blocking probe of a phase (test_wait): the first look of every wait.
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-#if WAN_MBAR_TEST_WAIT
         "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-#else
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-#endif
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
@@ -89,7 +82,8 @@ __device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity, u
 }
 
 // Wait for the phase with the given parity to complete.  Returns false on a
-// timeout (own or signalled through *abort by another warp of the CTA).
+// timeout (own or signalled through *abort by another warp of the CTA).  A
+// limit of 0 gives up as soon as a probe finds the phase still open.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           const WaitCtl& wc) {
     if (mbar_try(bar, parity)) return true;
@@ -97,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     while (true) {
         if (mbar_try_sleep(bar, parity, wc.limit_ns < 100000ull ? (uint32_t)wc.limit_ns : 100000u)) return true;
         if (*abort) return false;
-        if (global_ns() - t0 > wc.limit_ns) {
+        if (wc.limit_ns == 0 || global_ns() - t0 > wc.limit_ns) {
             *abort = 1;
             if (wc.err) atomicExch(wc.err, ERR_TIMEOUT);
             return false;
@@ -325,21 +319,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
     return y;
 }
-// 2^x for a pair through one MUFU instruction: x rounded to f16 (relative error
-// of 2^x <= |x| 2^-11 ln 2, 0.13 % at |x| = 8), ex2.approx.f16x2, widened back
-// to fp32.  Two exponentials per MUFU issue instead of one.
-__device__ __forceinline__ void ex2_f16x2(float x0, float x1, float& e0, float& e1) {
-    uint32_t h, e;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x1), "f"(x0));  // x0 in the low half
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-    asm("{\n\t.reg .b16 lo, hi;\n\t"
-        "mov.b32 {lo, hi}, %2;\n\t"
-        "cvt.f32.f16 %0, lo;\n\t"
-        "cvt.f32.f16 %1, hi;\n\t}"
-        : "=f"(e0), "=f"(e1)
-        : "r"(e));
-}
-
 // Packed fp32 pairs (two lanes of one 64-bit register) for the f32x2 ALU ops.
 __device__ __forceinline__ uint64_t f2pack(float a, float b) {
     uint64_t r;
@@ -368,34 +347,6 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
-}
-
-// 2^x for a pair of x <= 8 without the MUFU and without scalar FP32 or
-// integer-multiply work (which would compete with tcgen05.mma issue on the
-// same SM sub-partition): x = n + f with n the nearest integer (magic-number
-// rounding on packed f32x2 adds) and |f| <= 1/2; p(f) ~ 2^f from a cubic
-// fitted by weighted least squares on Chebyshev nodes (coefficients from
-// gen_exp2_poly.py, relative error < 8e-5), evaluated with packed FMAs; 2^n
-// built by inserting the biased exponent n + 127 (the low byte of the rounded
-// sum) into an empty word with bfi, applied with one packed multiply.  x is
-// clamped at -125 so the exponent never underflows (2^-125 ~ 2e-38 stands
-// in for 0).
-__device__ __forceinline__ void ex2_poly2(uint64_t x2, float& e0, float& e1) {
-    float x0, x1;
-    f2unpack(x2, x0, x1);
-    const uint64_t xc = f2pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-    const uint64_t magic = f2pack(12583039.0f, 12583039.0f);  // 1.5 * 2^23 + 127
-    const uint64_t t2 = add2(xc, magic);                        // low byte of the bits: n + 127
-    const uint64_t fr = sub2(xc, sub2(t2, magic));
-    uint64_t p2 = fma2(f2pack(5.508868396e-02f, 5.508868396e-02f), fr, f2pack(2.426040471e-01f, 2.426040471e-01f));
-    p2 = fma2(p2, fr, f2pack(6.932762265e-01f, 6.932762265e-01f));
-    p2 = fma2(p2, fr, f2pack(9.999289513e-01f, 9.999289513e-01f));
-    float t0, t1;
-    f2unpack(t2, t0, t1);
-    uint32_t s0, s1;
-    asm("bfi.b32 %0, %1, 0, 23, 8;" : "=r"(s0) : "r"(__float_as_uint(t0)));
-    asm("bfi.b32 %0, %1, 0, 23, 8;" : "=r"(s1) : "r"(__float_as_uint(t1)));
-    f2unpack(mul2(p2, f2pack(__uint_as_float(s0), __uint_as_float(s1))), e0, e1);
 }
 
 __device__ __forceinline__ float tanh_approx(float x) {

@@ -293,11 +293,19 @@ __global__ void __launch_bounds__(256) rmsnorm_rope_qk_kernel(__nv_bfloat16* buf
     }
 }
 
+bool rmsnorm_rope_shape_ok(int D, long long ld) {
+    if (D <= 0 || D % 256 || ld % 8 || ld < D) return false;
+    switch (D / 256) {
+        case 1: case 2: case 3: case 4: case 6: case 8: case 12: case 16: case 20: case 24: return true;
+        default: return false;
+    }
+}
+
 cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float eps, const float* gains,
                                 long long gain_stride, int nseg, long long seg_stride, const RopeTables* rope,
                                 int rope_L, const LaunchCtx& ctx) {
     if (rows <= 0 || nseg <= 0) return cudaSuccess;
-    if (D % 256 || ld % 8 || seg_stride % 8) return cudaErrorInvalidValue;
+    if (!rmsnorm_rope_shape_ok(D, ld) || seg_stride % 8) return cudaErrorInvalidValue;
     RopeTables rt{};
     int use_rope = 0;
     if (rope) {

@@ -322,13 +322,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int kblocks = p.K / Cfg::BK;
+    // producer: stages with a load issued and the phase it completes; MMA issuer:
+    // whether any MMA went out (both drained after an abort, before the CTA exits)
+    uint32_t armed = 0, armed_par = 0;
+    bool issued = false;
 
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer ----------------
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t armed = 0, armed_par = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
                 int mb, nb;
@@ -349,10 +352,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     }
                 }
             }
-            if (!ok) {  // drain the loads still in flight before the CTA exits
-                for (int s = 0; s < STAGES; ++s)
-                    if (armed & (1u << s)) mbar_drain(full + s, (armed_par >> s) & 1u, 200000000ull);
-            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -362,7 +361,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            bool ok = true, issued = false;
+            bool ok = true;
             for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
                 if (!mbar_wait(tempty + acc, acc_phase ^ 1, abort_flag, p.wc)) {
                     ok = false;
@@ -394,10 +393,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 umma_commit(tfull + acc);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
-            }
-            if (!ok && issued) {  // let the tensor core finish before TMEM is freed
-                umma_commit(drain);
-                mbar_drain(drain, 0, 200000000ull);
             }
         }
     } else {
@@ -431,6 +426,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
 
     __syncthreads();
+    if (*abort_flag && lane == 0) {
+        // a wait gave up somewhere in the CTA: let this CTA's own loads and MMAs
+        // land (bounded) before its shared and tensor memory are released
+        if (warp == 0) {
+            for (int s = 0; s < STAGES; ++s)
+                if (armed & (1u << s)) mbar_drain(full + s, (armed_par >> s) & 1u, 200000000ull);
+        } else if (warp == 1 && issued) {
+            umma_commit(drain);
+            mbar_drain(drain, 0, 200000000ull);
+        }
+    }
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();

@@ -77,6 +77,10 @@ struct RopeTables {
     int nt, nh, nw;   // pairs per axis
 };
 
+// Row widths and strides the RMSNorm kernels take: D a supported multiple of
+// 256 (up to 6144), ld a multiple of 8 elements and >= D.
+bool rmsnorm_rope_shape_ok(int D, long long ld);
+
 // In-place RMSNorm (+ RoPE) of nseg row segments (segment s at column
 // s * seg_stride, gain gains + s * gain_stride).
 cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float eps, const float* gains,

@@ -78,6 +78,16 @@ extern "C" wan_status wan_op_rmsnorm_rope_noalloc(void* buf, int64_t ld, int row
                                                   float theta, void* stream) {
     using namespace wan;
     if (!buf || !gain) return WAN_EINVAL;
+    // every shape check comes before the table is touched or anything is launched
+    if (!rmsnorm_rope_shape_ok(D, ld)) return WAN_ESHAPE;
+    if (rope && (Fp <= 0 || Hp <= 0 || Wp <= 0 || rope_t % 2 || rope_h % 2 || rope_w % 2 ||
+                 rope_t + rope_h + rope_w != 128 || !(theta > 0.f)))
+        return WAN_ESHAPE;
+    // the fixed table holds kMaxRopePositions positions per axis
+    if (rope && (Fp > kMaxRopePositions || Hp > kMaxRopePositions || Wp > kMaxRopePositions)) return WAN_ESHAPE;
+    if (rows <= 0) return WAN_OK;
+    // an error already pending on this thread is the caller's: report it, launch nothing
+    if (cudaPeekAtLastError() != cudaSuccess) return WAN_ECUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess) return WAN_ECUDA;
@@ -87,18 +97,13 @@ extern "C" wan_status wan_op_rmsnorm_rope_noalloc(void* buf, int64_t ld, int row
         cudaError_t e = launch_rmsnorm_rope(buf, ld, rows, D, eps, gain, 0, 1, 0, nullptr, 0, ctx);
         return e == cudaSuccess ? WAN_OK : (e == cudaErrorInvalidValue ? WAN_ESHAPE : WAN_ECUDA);
     }
-    if (Fp <= 0 || Hp <= 0 || Wp <= 0 || rope_t % 2 || rope_h % 2 || rope_w % 2 || rope_t + rope_h + rope_w != 128 ||
-        !(theta > 0.f))
-        return WAN_ESHAPE;
-    // the fixed table holds kMaxRopePositions positions per axis
-    if (Fp > kMaxRopePositions || Hp > kMaxRopePositions || Wp > kMaxRopePositions) return WAN_ESHAPE;
     float2* tab = table_address();
     if (!tab) return WAN_ECUDA;
     const int nt = rope_t / 2, nh = rope_h / 2, nw = rope_w / 2;
     const int total = Fp * nt + Hp * nh + Wp * nw;
     fill_rope_table<<<(total + 255) / 256, 256, 0, st>>>(tab, Fp, Hp, Wp, rope_t, rope_h, rope_w,
                                                          std::log((double)theta));
-    if (cudaGetLastError() != cudaSuccess) return WAN_ECUDA;
+    if (cudaPeekAtLastError() != cudaSuccess) return WAN_ECUDA;
     RopeTables rt{tab, tab + (size_t)Fp * nt, tab + (size_t)Fp * nt + (size_t)Hp * nh, Fp, Hp, Wp, nt, nh, nw};
     cudaError_t e = launch_rmsnorm_rope(buf, ld, rows, D, eps, gain, 0, 1, 0, &rt, Fp * Hp * Wp, ctx);
     return e == cudaSuccess ? WAN_OK : (e == cudaErrorInvalidValue ? WAN_ESHAPE : WAN_ECUDA);

@@ -1017,8 +1017,14 @@ wan_status wan_op_rmsnorm_rope(void* buf, int64_t ld, int rows, int D, float eps
     int nt, nh, nw;
     rope_tables_host(c, Fp, Hp, Wp, tab, nt, nh, nw);
     float2* d = nullptr;
-    if (cudaMalloc(&d, tab.size() * sizeof(float2)) != cudaSuccess) return WAN_ENOMEM;
-    cudaMemcpy(d, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
+    if (cudaMalloc(&d, tab.size() * sizeof(float2)) != cudaSuccess) {
+        cudaGetLastError();
+        return WAN_ENOMEM;
+    }
+    if (cudaMemcpy(d, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaFree(d);
+        return WAN_ECUDA;
+    }
     wan::RopeTables rt{d, d + (size_t)Fp * nt, d + (size_t)Fp * nt + (size_t)Hp * nh, Fp, Hp, Wp, nt, nh, nw};
     cudaError_t e = wan::launch_rmsnorm_rope(buf, ld, rows, D, eps, gain, 0, 1, 0, &rt, Fp * Hp * Wp, ctx);
     cudaStreamSynchronize(ctx.stream);
