@@ -250,8 +250,12 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     ms = e0.elapsed_time(e1) / args.steps
+    from video_diffusion_transformer_dit_b200.binding import BLOCK_GEMMS
     kt = {c: dit.kernel_time(c) for c in ("self_attention", "gemm", "cross_attention", "layernorm",
-                                         "rmsnorm_rope", "patchify", "embedding")}
+                                         "rmsnorm_rope", "patchify", "embedding") + BLOCK_GEMMS}
+    gemm_parts = {c: kt.pop(c) for c in BLOCK_GEMMS}
+    kt["gemm"] = (kt["gemm"][0] + sum(v[0] for v in gemm_parts.values()),
+                  kt["gemm"][1] + sum(v[1] for v in gemm_parts.values()))
     launches = dit.last_launch_count()
     dit.set_option(WAN_OPT_KERNEL_TIMING, 0)
 
@@ -317,6 +321,7 @@ def run_ours(args, rank, world, local_rank):
                      if args.workload == DEFAULT_WORKLOAD else None,
                      "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
         "kernel_ms_per_step": {c: v[0] for c, v in kt.items()},
+        "gemm_ms_per_step": {c: v[0] for c, v in gemm_parts.items()},
         "e2e": {"value": whole_job_tokens_per_s(world, B, L, ms_e2e), "unit": "tokens/s", "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches * args.steps,
@@ -327,7 +332,57 @@ def run_ours(args, rank, world, local_rank):
 
 # ---------------------------------------------------------------- single-kernel mode
 KERNELS = ("self_attention", "cross_attention", "gemm_qkv", "gemm_o", "gemm_ffn_up", "gemm_ffn_down", "layernorm",
-           "rmsnorm_rope")
+           "rmsnorm_rope", "vae_conv", "vae_decode")
+
+
+def run_vae(args):
+    """Time the Wan2.1 VAE decoder's implicit-GEMM convolution (384 -> 384,
+    3x3x3, 2-frame cache, 2 frames at 120x208: the shape of up block 1 at 480p)
+    or a whole decode of the 480p latent (21 frames 60x104 -> 81 frames
+    480x832), random weights."""
+    import torch
+    from video_diffusion_transformer_dit_b200 import binding as Bd
+    from video_diffusion_transformer_dit_b200 import build
+    build.build()
+    dev = "cuda"
+    g = torch.Generator(device=dev).manual_seed(0)
+    if args.kernel == "vae_conv":
+        Ci = Co = 384
+        T, H, W = 2, 120, 208
+        x = torch.randn(1, T, H, W, Ci, generator=g, device=dev).to(torch.bfloat16)
+        cache = torch.randn(1, 2, H, W, Ci, generator=g, device=dev).to(torch.bfloat16)
+        w = (torch.randn(Co, 27 * Ci, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        bias = torch.zeros(Co, device=dev)
+        y = torch.empty(1, T, H, W, Co, dtype=torch.bfloat16, device=dev)
+        fn = lambda: Bd.op_conv3d(x, w, bias, y, (3, 3, 3), Co, cache=cache)
+        work, unit = 2.0 * T * H * W * Co * 27 * Ci, "TFLOP/s"
+        sync = Bd.op_sync
+    else:
+        from video_diffusion_transformer_dit_b200 import synth
+        vae = Bd.WanVAE(max_batch=1, max_h=60, max_w=104)
+        vae.load_weights(synth.make_vae_weights(seed=0, device=dev))
+        z = torch.randn(1, 16, 21, 60, 104, generator=g, device=dev)
+        video = torch.empty(1, 3, 81, 480, 832, device=dev)
+        fn = lambda: vae.decode(z, video=video)
+        work, unit = 81.0, "frames/s"
+        sync = lambda: vae._check(Bd.lib().wan_vae_sync(vae._h, Bd._stream(None)))
+    for _ in range(args.warmup):
+        fn()
+    sync()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    sync()
+    ms = e0.elapsed_time(e1) / args.steps
+    rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1.0)
+    out = {"kernel": args.kernel, "avg_ms": ms, "achieved": rate, "unit": unit, "launches": args.steps}
+    if unit == "TFLOP/s":
+        peaks = load_peaks()
+        out.update(peak=peaks["bf16_tflops"], frac=rate / peaks["bf16_tflops"], peak_source=peaks["source"] + " (burst)")
+    print(json.dumps(out))
+    return 0
 
 
 def run_kernel(args):
@@ -421,6 +476,8 @@ def main():
     ap.add_argument("--kernel", choices=KERNELS, default=None,
                     help="time one kernel alone at the workload's shapes (profiling aid)")
     args = ap.parse_args()
+    if args.kernel in ("vae_conv", "vae_decode"):
+        return run_vae(args)
     if args.kernel:
         return run_kernel(args)
 

@@ -161,6 +161,77 @@ WANDIT_API wan_status wan_dit_forward_image(wan_dit* h, const void* latent, int 
                            const void* image, int Li,
                            float* velocity, int io_on_device, void* stream);
 
+/* One flow-matching sampler step of a classifier-free-guided run, fused into
+ * the forward ("【VLA与模仿学习】Wan2.1框架与训练源码导读" §7: the CFG combination
+ * v = v_u + s (v_c - v_u) of the conditional and unconditional predictions and
+ * the Euler update x_next = x + (sigma_next - sigma) v; the flow-shifted noise
+ * levels come from wan_flow_sigmas).  Runs the B = 2 forward of the same
+ * latent with two contexts and, in the proj_out epilogue, combines each
+ * token's two velocity rows (each rounded to bf16, as wan_dit_forward returns
+ * them) and writes the updated latent -- the two velocities never reach memory.
+ *   x         float [1, in_ch, F, Hz, Wz] sampler state (the latent)
+ *   timestep  the DiT timestep of this step (both samples)
+ *   context   bf16 [2, Lc, text_dim]: row block 0 the conditional prompt,
+ *             row block 1 the unconditional (negative) prompt
+ *   guidance  s; sigma, sigma_next: this step's and the next noise level
+ *   x_next    float [1, out_ch, F, Hz, Wz] output; may alias x
+ * x, context and x_next are device pointers when io_on_device != 0, else host
+ * pointers (copies inside the call, in stream order).  The result equals
+ * wan_dit_forward at B = 2 followed by wan_op_cfg_euler on its two halves, bit
+ * for bit.  Needs in_ch == out_ch (WAN_EUNSUPPORTED otherwise, e.g. I2V) and
+ * max_batch >= 2; other limits as wan_dit_forward.                          */
+WANDIT_API wan_status wan_dit_forward_cfg_euler(wan_dit* h, const float* x, int F, int Hz, int Wz,
+                           float timestep, const void* context, int Lc,
+                           float guidance, float sigma, float sigma_next,
+                           float* x_next, int io_on_device, void* stream);
+
+/* Noise levels of a `steps`-step flow-matching run, steps + 1 doubles from 1
+ * down to a final 0: the uniform ladder u_i = 1 - i/steps (i < steps) under
+ * the flow shift  sigma = shift u / (1 + (shift - 1) u),  which multiplies the
+ * noise odds u / (1 - u) by `shift` (the pswp.cn WanPipeline notes set
+ * flow_shift 3.0 for 480p and 5.0 for 720p in the scheduler; "读完 Wan2.2 全部源码之后"
+ * §"shift 参数生效了两次,在两个地方": it takes effect where the timesteps are
+ * set).  The DiT timestep of step i is sigmas[i] * num_train_timesteps.  Pure
+ * host function; WAN_EINVAL for steps < 1, shift <= 0 or sigmas == NULL.    */
+WANDIT_API wan_status wan_flow_sigmas(int steps, double shift, double* sigmas);
+
+/* Sequence-parallel (Ulysses) forward, one rank's part ("读完 Wan2.2 全部源码之后",
+ * §"显存和算力怎么分": q, k, v are scattered along heads and gathered along the
+ * sequence by an all-to-all, every rank runs attention over the whole
+ * sequence for its heads, and a second all-to-all brings the outputs back).
+ * The tokens are split into `world` shards of Ls = ceil(L / world) tokens;
+ * rank r holds global tokens [r * Ls, (r + 1) * Ls), the last shard padded
+ * past L.  Padding is explicit, so no shard is shorter than the others (the
+ * uneven torch.chunk split those pages warn about cannot occur): padding
+ * tokens never act as keys (the attention masks keys >= L) and their outputs
+ * are dropped; RoPE and the timestep use each token's global position.
+ * Everything except self-attention is token-local and runs on the shard.
+ * The caller moves the exchange buffers between ranks (e.g. NCCL
+ * all_to_all_single per sample); the library reads and writes only this
+ * rank's device memory.  Call order per forward:
+ *   sp_begin; for block i: sp_block_qkv(i) -> exchange -> sp_attention ->
+ *   exchange back -> sp_block_finish(i); sp_end.
+ * Layouts (bf16, device, hd = 128 * heads / world):
+ *   send   [B][world][Ls][3][hd]  q, k, v of this shard, head group j in slot j
+ *          (q and k RMSNorm'd across all heads and rotated)
+ *   recv   [B][world][Ls][3][hd]  = [B][Lp][3 hd]: this rank's head group for
+ *          every token of the padded sequence (Lp = world * Ls)
+ *   out    [B][Lp][hd]            attention output of this rank's heads
+ *   back   [B][world][Ls][hd]     slot j: head group j's output for this shard
+ * sp_begin takes the whole latent, the whole timestep ([B] or [B, L]) and the
+ * context, host or device like wan_dit_forward; it needs heads % world == 0,
+ * Ls <= max_tokens and a text-to-video model.  sp_end writes the full-size
+ * velocity [B, out_ch, F, Hz, Wz] holding this shard's tokens and zeros
+ * elsewhere: the sum over ranks is the velocity.  Calls are eager (no graph)
+ * and asynchronous on `stream`; out-of-order calls return WAN_EINVAL.       */
+WANDIT_API wan_status wan_dit_sp_begin(wan_dit* h, const void* latent, int latent_dtype,
+                           int B, int F, int Hz, int Wz, const float* timestep, int per_token,
+                           const void* context, int Lc, int rank, int world, int io_on_device, void* stream);
+WANDIT_API wan_status wan_dit_sp_block_qkv(wan_dit* h, int block, void* send, void* stream);
+WANDIT_API wan_status wan_dit_sp_attention(wan_dit* h, const void* recv, void* out, void* stream);
+WANDIT_API wan_status wan_dit_sp_block_finish(wan_dit* h, int block, const void* back, void* stream);
+WANDIT_API wan_status wan_dit_sp_end(wan_dit* h, float* velocity, int io_on_device, void* stream);
+
 /* Expert of the Wan2.2 A14B two-expert route for one sampling step: 0 (the
  * high-noise expert) when t >= boundary * num_train_timesteps, else 1 (the
  * low-noise expert).  One expert runs the whole step, both CFG forwards
@@ -184,10 +255,16 @@ WANDIT_API wan_status wan_dit_set_block_dump(wan_dit* h, void* dst);
  * the forward, read back with wan_dit_kernel_time; default 0).            */
 enum { WAN_OPT_GRAPH = 1, WAN_OPT_WAIT_LIMIT_NS = 2, WAN_OPT_KERNEL_TIMING = 3 };
 
-/* Kernel classes of the forward, for wan_dit_kernel_time(). */
+/* Kernel classes of the forward, for wan_dit_kernel_time().  WAN_KC_GEMM
+ * covers the GEMMs outside the blocks (patch, timestep, text, cross K/V,
+ * proj_out); the block GEMMs have a class each: q/k/v projection (with the
+ * q/k RMSNorm epilogue), attention output, cross-attention query and output,
+ * FFN up and down.                                                          */
 enum {
     WAN_KC_PATCHIFY = 0, WAN_KC_GEMM = 1, WAN_KC_SELF_ATTENTION = 2, WAN_KC_CROSS_ATTENTION = 3,
-    WAN_KC_LAYERNORM = 4, WAN_KC_RMSNORM_ROPE = 5, WAN_KC_EMBEDDING = 6, WAN_KC_COUNT = 7
+    WAN_KC_LAYERNORM = 4, WAN_KC_RMSNORM_ROPE = 5, WAN_KC_EMBEDDING = 6,
+    WAN_KC_GEMM_QKV = 7, WAN_KC_GEMM_O = 8, WAN_KC_GEMM_Q2 = 9, WAN_KC_GEMM_O2 = 10,
+    WAN_KC_GEMM_FFN_UP = 11, WAN_KC_GEMM_FFN_DOWN = 12, WAN_KC_COUNT = 13
 };
 
 /* With WAN_OPT_KERNEL_TIMING on: total device time (ms) and number of

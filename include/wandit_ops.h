@@ -33,14 +33,24 @@ extern "C" {
  *  WAN_EPI_BIAS_F32      out f32  = acc + bias[c]
  *  WAN_EPI_UNPATCHIFY    velocity f32 = bf16(acc + bias[c]) scattered by the unpatchify map
  *                        (WanTransformer3DModel step 5); row r = b * L + token, column
- *                        c = ((kt * ph + kh) * pw + kw) * up_C + ch.                      */
+ *                        c = ((kt * ph + kh) * pw + kw) * up_C + ch.
+ *  WAN_EPI_QK_NORM       the q/k projection with "qk_norm = rms_norm_across_heads" split
+ *                        in two: for c < norm_cols, out bf16 = gain[c] * (acc + bias[c]),
+ *                        rotated by the 3-axis RoPE of token r % (rope_F*rope_H*rope_W)
+ *                        when rope != 0, and ssq[r * ssq_ld + c / 128] = sum over the
+ *                        128-column group of (acc + bias)^2 (fp32); columns >= norm_cols
+ *                        get the bias epilogue.  The row factor rsqrt(sum / D + eps)
+ *                        commutes with the gain and the rotation and is applied by
+ *                        wan_op_rms_apply (keys) or wan_op_attention_qnorm (queries).
+ *                        N % 256 == 0, norm_cols % 128 == 0.                            */
 enum {
     WAN_EPI_BIAS = 0,
     WAN_EPI_BIAS_GELU = 1,
     WAN_EPI_GATE_RESIDUAL = 2,
     WAN_EPI_RESIDUAL = 3,
     WAN_EPI_BIAS_F32 = 4,
-    WAN_EPI_UNPATCHIFY = 5
+    WAN_EPI_UNPATCHIFY = 5,
+    WAN_EPI_QK_NORM = 8
 };
 
 typedef struct {
@@ -55,6 +65,15 @@ typedef struct {
     int mod_div;          /* modulation row = r / mod_div                         */
     int64_t mod_ld;       /* row stride of gate1 in elements                      */
     int up_C, up_F, up_Hz, up_Wz; /* unpatchify geometry, patch (1,2,2)           */
+    /* WAN_EPI_QK_NORM only: */
+    const float* gain;    /* [norm_cols] f32 RMSNorm gains                         */
+    float* ssq;           /* f32 [M, ssq_ld] per-128-column sums of squares (output) */
+    int64_t ssq_ld;       /* row stride of ssq, >= norm_cols / 128                  */
+    int norm_cols;        /* leading columns that are normed                       */
+    int rope;             /* 1: rotate the normed columns (RoPE), 0: no rotation     */
+    int rope_F, rope_H, rope_W;   /* post-patch grid of the RoPE positions         */
+    int rope_t, rope_h, rope_w;   /* head-dim split (even, sum 128)                */
+    float rope_theta;     /* RoPE base                                             */
 } wan_epilogue;
 
 /* C = epilogue(A[M,K] . W[N,K]^T).  A, W bf16 device pointers, 16-byte aligned
@@ -72,6 +91,22 @@ WANDIT_API wan_status wan_op_gemm(const void* A, int64_t lda, const void* W, int
 WANDIT_API wan_status wan_op_attention(const void* q, int64_t ldq, const void* k, int64_t ldk,
                             const void* v, int64_t ldv, void* o, int64_t ldo,
                             int B, int heads, int Lq, int Lk, void* stream);
+
+/* wan_op_attention with unnormalised queries: each query row (b, l) is first
+ * multiplied by its RMSNorm factor rsqrt(sum_{g < ngroups} q_ssq[(b * Lq + l) *
+ * ssq_ld + g] / (128 * heads) + eps), the sums of squares coming from the
+ * WAN_EPI_QK_NORM epilogue (RMSNorm across heads: "qk_norm =
+ * rms_norm_across_heads").  Same layouts and limits as wan_op_attention.     */
+WANDIT_API wan_status wan_op_attention_qnorm(const void* q, int64_t ldq, const void* k, int64_t ldk,
+                            const void* v, int64_t ldv, void* o, int64_t ldo,
+                            int B, int heads, int Lq, int Lk,
+                            const float* q_ssq, int64_t ssq_ld, int ngroups, float eps, void* stream);
+
+/* In-place row factor of the split RMSNorm: buf[r, 0:D) *= rsqrt(sum_{g <
+ * ngroups} ssq[r * ssq_ld + g] / D + eps) for bf16 rows (row stride ld); the
+ * key half of WAN_EPI_QK_NORM.  D as for wan_op_rmsnorm_rope.               */
+WANDIT_API wan_status wan_op_rms_apply(void* buf, int64_t ld, int rows, int D, const float* ssq, int64_t ssq_ld,
+                                       int ngroups, float eps, void* stream);
 
 /* LayerNorm of bf16 rows x[rows, D] (fp32 statistics, biased variance, eps),
  * then either an affine (gamma, beta; mode 1: norm2) or the adaLN modulation

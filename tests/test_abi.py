@@ -19,7 +19,7 @@ def lib():
 
 def declared_symbols():
     names = set()
-    for h in ("wandit.h", "wandit_ops.h"):
+    for h in ("wandit.h", "wandit_ops.h", "wanvae.h"):
         text = open(os.path.join(ROOT, "include", h)).read()
         names |= set(re.findall(r"WANDIT_API\s+[\w\s\*]+?\b(wan_\w+)\s*\(", text))
     return names
@@ -75,3 +75,16 @@ def test_null_handle_calls_are_refused(lib):
     assert lib.wan_dit_sync(None, None) == 1
     assert lib.wan_dit_last_launch_count(None) == 0
     assert lib.wan_dit_last_error(None) == b"null handle"
+
+
+def test_flow_sigmas_match_oracle(lib):
+    """The host-side sigma schedule against the oracle's reading R22."""
+    import torch
+    from oracle import wan_oracle as O
+    from video_diffusion_transformer_dit_b200 import binding
+    for steps, shift in ((1, 1.0), (4, 1.0), (50, 3.0), (40, 5.0), (30, 0.5)):
+        got = torch.tensor(binding.flow_sigmas(steps, shift), dtype=torch.float64)
+        torch.testing.assert_close(got, O.sampling_sigmas(steps, shift), rtol=1e-14, atol=1e-15)
+    for steps, shift in ((0, 3.0), (10, 0.0), (10, -1.0)):
+        with pytest.raises(binding.WanError):
+            binding.flow_sigmas(steps, shift)

@@ -364,3 +364,86 @@ def test_forward_5b_per_token_30_blocks_properties():
     27280 tokens, per-token timesteps (first latent frame clean), 30 blocks."""
     n = _full_depth_properties("wan5b-121f-704x1280-pertoken", seed=10)
     assert n > 10 * 30
+
+
+# ---------------------------------------------------------------- sampler step fused into proj_out (CFG + Euler)
+
+def _cfg_case(name, seed, num_blocks=None):
+    from video_diffusion_transformer_dit_b200 import configs, synth
+    w = configs.workload(name)
+    cfg = dict(w["cfg"])
+    if num_blocks is not None:
+        cfg["num_blocks"] = num_blocks
+    _, Cc, F, Hz, Wz = w["latent"]
+    Lc = w["text_len"]
+    W = synth.make_weights(cfg, seed=seed)
+    x = synth.make_latent((1, Cc, F, Hz, Wz), seed=seed)
+    ctx = synth.make_context(2, Lc, cfg["text_dim"], seed=seed)      # conditional, unconditional
+    return cfg, W, x, ctx
+
+
+def test_forward_cfg_euler_one_block_against_oracle():
+    """x_next = x + (sigma_next - sigma)(v_u + s (v_c - v_u)) with the two
+    velocities of the B = 2 forward (same latent, conditional and unconditional
+    context), one block + head, a step of the 50-step 480p schedule (shift 3)."""
+    from video_diffusion_transformer_dit_b200 import binding as Bd
+    cfg, W, x, ctx = _cfg_case("wan1.3b-1blk-3x16x16", seed=12)
+    _, Cc, F, Hz, Wz = x.shape
+    L, Lc = O.token_count(F, Hz, Wz), ctx.shape[1]
+    sig = Bd.flow_sigmas(50, 3.0)
+    i, s = 10, 5.0
+    t = float(torch.tensor(sig[i] * 1000.0, dtype=torch.float32))
+    dit = make_dit(cfg, 2, L, Lc, W)
+    xn = dit.forward_cfg_euler(x.cuda(), t, ctx.cuda(), s, sig[i], sig[i + 1], sync=True).cpu()
+    xd = x.to(DT)
+    v = O.forward(xd.expand(2, -1, -1, -1, -1), torch.full((2,), t, dtype=DT), ctx.to(DT), to64(W), cfg)
+    ref = O.euler_step(xd, sig[i], sig[i + 1], O.cfg_combine(v[1:2], v[0:1], s))
+    ds = sig[i + 1] - sig[i]
+    err = rel_l2((xn.to(DT) - xd) / ds, (ref - xd) / ds)          # the update carries the model output
+    print(f"\n[CFG+Euler 1 block] update rel-L2 {err:.3e}")
+    assert err < TOL
+    # the unfused path (B = 2 forward, then the sampler-step op) gives the same bits
+    vel = dit.forward(x.expand(2, -1, -1, -1, -1).contiguous().cuda(), torch.full((2,), t).cuda(), ctx.cuda(),
+                      sync=True)
+    out = torch.empty_like(x).cuda()
+    Bd.op_cfg_euler(x.cuda(), vel[0:1].contiguous(), vel[1:2].contiguous(), s, sig[i], sig[i + 1], out)
+    Bd.op_sync()
+    assert torch.equal(out.cpu(), xn)
+    # host buffers, and x_next aliasing x
+    xh = dit.forward_cfg_euler(x.pin_memory(), t, ctx.pin_memory(), s, sig[i], sig[i + 1])
+    dit.sync()
+    assert torch.equal(xh, xn)
+    xa = x.clone().cuda()
+    dit.forward_cfg_euler(xa, t, ctx.cuda(), s, sig[i], sig[i + 1], x_next=xa, sync=True)
+    assert torch.equal(xa.cpu(), xn)
+
+
+def test_forward_cfg_euler_480p_30_blocks_matches_unfused():
+    """The 480p CFG pair (L = 32760, 30 blocks): fused sampler step bit-identical
+    to the B = 2 forward followed by the separate sampler-step kernel, at two
+    steps of the schedule (the per-call scalars change without a new capture)."""
+    from video_diffusion_transformer_dit_b200 import binding as Bd
+    from video_diffusion_transformer_dit_b200 import synth
+    cfg, _, x, ctx = _cfg_case("wan1.3b-81f-480x832-cfg2", seed=13, num_blocks=1)
+    cfg["num_blocks"] = 30
+    W = synth.make_weights(cfg, seed=13, device="cuda")
+    _, Cc, F, Hz, Wz = x.shape
+    L, Lc = O.token_count(F, Hz, Wz), ctx.shape[1]
+    dit = make_dit(cfg, 2, L, Lc)
+    dit.load_weights(W)
+    del W
+    sig = Bd.flow_sigmas(50, 3.0)
+    xc, cc = x.cuda(), ctx.cuda()
+    launches = None
+    for i in (0, 37):
+        t = float(torch.tensor(sig[i] * 1000.0, dtype=torch.float32))
+        xn = dit.forward_cfg_euler(xc, t, cc, 5.0, sig[i], sig[i + 1], sync=True)
+        launches = dit.last_launch_count()
+        vel = dit.forward(xc.expand(2, -1, -1, -1, -1).contiguous(), torch.full((2,), t).cuda(), cc, sync=True)
+        out = torch.empty_like(xc)
+        Bd.op_cfg_euler(xc, vel[0:1].contiguous(), vel[1:2].contiguous(), 5.0, sig[i], sig[i + 1], out)
+        Bd.op_sync()
+        assert torch.isfinite(xn).all()
+        assert torch.equal(out, xn), i
+        assert not torch.equal(xn, xc)
+    assert launches == dit.last_launch_count()

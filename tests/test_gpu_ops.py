@@ -268,6 +268,49 @@ def test_rmsnorm_rope(rope):
     assert torch.equal(got[:, :D], buf[:, :D]) and torch.equal(got[:, 2 * D:], buf[:, 2 * D:])
 
 
+# ------------------------------------------------------------------ q/k RMSNorm split across the QKV epilogue
+@pytest.mark.parametrize("rope", [True, False])
+def test_qk_norm_epilogue_row_factors_and_attention(rope):
+    """The self-attention path with RMSNorm across heads in two parts: the QKV
+    GEMM epilogue (gain, RoPE, per-head sums of squares), the key row factors in
+    place, the query row factors inside the attention -- against the oracle's
+    RMSNorm + RoPE + attention.  B = 2, L = 135 tokens (a ragged second tile)."""
+    Fp, Hp, Wp = 3, 5, 9
+    L, Bn, D, h, eps = Fp * Hp * Wp, 2, 1536, 12, 1e-6
+    R = Bn * L
+    g = torch.Generator().manual_seed(40)
+    y = torch.randn(R, D, generator=g).to(torch.bfloat16)
+    W = (0.02 * torch.randn(3 * D, D, generator=g)).to(torch.bfloat16)
+    bias = 0.02 * torch.randn(3 * D, generator=g)
+    gain = 1 + 0.1 * torch.randn(2 * D, generator=g)
+    qkv = torch.empty(R, 3 * D, dtype=torch.bfloat16, device="cuda")
+    ssq = torch.empty(R, 2 * h, device="cuda")
+    B().op_gemm(y.cuda(), W.cuda(), "qk_norm", qkv, bias=bias.cuda(), gain=gain.cuda(), ssq=ssq, norm_cols=2 * D,
+                rope_grid=(Fp, Hp, Wp) if rope else None)
+    B().op_sync()
+    lin = O.linear(y.to(DT), W.to(DT), bias.to(DT))
+    ref_ssq = (lin[:, :2 * D] ** 2).reshape(R, 2 * h, 128).sum(-1)
+    assert rel_l2(ssq.cpu(), ref_ssq) < 1e-4
+    ang = O.rope_angles((Fp, Hp, Wp), (44, 42, 42), 10000.0)
+
+    def rot(x):
+        return O.rope_apply(x.reshape(Bn, L, h, 128), ang).reshape(R, D) if rope else x
+    # stored q and k: gain * (acc + bias), rotated, not yet normalised; v plain
+    stored = qkv.cpu()
+    assert rel_l2(stored[:, :D], rot(lin[:, :D] * gain[:D].to(DT))) < TOL
+    assert rel_l2(stored[:, 2 * D:], lin[:, 2 * D:]) < TOL
+    base = qkv.data_ptr()
+    B().op_rms_apply(base + 2 * D, 3 * D, R, D, ssq.data_ptr() + 4 * h, ssq.stride(0), h, eps)
+    o = torch.empty(R, D, dtype=torch.bfloat16, device="cuda")
+    B().op_attention_qnorm(base, 3 * D, base + 2 * D, 3 * D, base + 4 * D, 3 * D, o, Bn, h, L, L, ssq, h, eps)
+    B().op_sync()
+    q = rot(O.rms_norm(lin[:, :D], eps, gain[:D].to(DT)))
+    k = rot(O.rms_norm(lin[:, D:2 * D], eps, gain[D:].to(DT)))
+    assert rel_l2(qkv.cpu()[:, D:2 * D], k) < TOL                     # keys normalised in place
+    ref = O.attention(q.reshape(Bn, L, h, 128), k.reshape(Bn, L, h, 128), lin[:, 2 * D:].reshape(Bn, L, h, 128))
+    assert rel_l2(o.cpu(), ref.reshape(R, D)) < TOL
+
+
 # ------------------------------------------------------------------ sampler step (CFG + Euler)
 def test_cfg_euler_matches_oracle_and_worked_example():
     g = torch.Generator().manual_seed(21)

@@ -168,3 +168,9 @@ def test_output_is_clamped():
     out = V.decode(torch.randn(1, 16, 2, 2, 2, dtype=DT) * 3, W, base=8)
     assert out.min() >= lo and out.max() <= hi
     assert (out.abs() == 1.0).any()                                                 # the clamp is active here
+
+
+def test_generator_table_matches_oracle_table():
+    from video_diffusion_transformer_dit_b200 import synth
+    assert synth.vae_param_shapes() == V.param_shapes()
+

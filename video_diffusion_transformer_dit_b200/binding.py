@@ -21,8 +21,10 @@ WAN_STATUS = {0: "WAN_OK", 1: "WAN_EINVAL", 2: "WAN_ESHAPE", 3: "WAN_ENOMEM", 4:
 WAN_DTYPE_F32, WAN_DTYPE_BF16 = 0, 1
 WAN_OPT_GRAPH, WAN_OPT_WAIT_LIMIT_NS, WAN_OPT_KERNEL_TIMING = 1, 2, 3
 KERNEL_CLASSES = {"patchify": 0, "gemm": 1, "self_attention": 2, "cross_attention": 3, "layernorm": 4,
-                  "rmsnorm_rope": 5, "embedding": 6}
-EPI = {"bias": 0, "bias_gelu": 1, "gate_residual": 2, "residual": 3, "bias_f32": 4, "unpatchify": 5}
+                  "rmsnorm_rope": 5, "embedding": 6, "gemm_qkv": 7, "gemm_o": 8, "gemm_q2": 9, "gemm_o2": 10,
+                  "gemm_ffn_up": 11, "gemm_ffn_down": 12}
+BLOCK_GEMMS = ("gemm_qkv", "gemm_o", "gemm_q2", "gemm_o2", "gemm_ffn_up", "gemm_ffn_down")
+EPI = {"bias": 0, "bias_gelu": 1, "gate_residual": 2, "residual": 3, "bias_f32": 4, "unpatchify": 5, "qk_norm": 8}
 
 # every symbol include/*.h declares
 SYMBOLS = ["wan_dit_create", "wan_dit_load_weights", "wan_dit_missing_weights", "wan_dit_forward", "wan_dit_sync",
@@ -31,7 +33,11 @@ SYMBOLS = ["wan_dit_create", "wan_dit_load_weights", "wan_dit_missing_weights", 
            "wan_dit_last_error", "wan_status_string", "wan_dit_destroy",
            "wan_op_gemm", "wan_op_attention", "wan_op_layernorm", "wan_op_rmsnorm_rope", "wan_op_patchify",
            "wan_op_unpatchify", "wan_op_sync", "wan_op_set_wait_limit_ns", "wan_op_rmsnorm_rope_noalloc", "wan_op_cfg_euler",
-           "wan_op_wait_selftest", "wan_op_causal_conv3d"]
+           "wan_op_wait_selftest", "wan_op_causal_conv3d", "wan_dit_forward_cfg_euler", "wan_flow_sigmas",
+           "wan_op_attention_qnorm", "wan_op_rms_apply", "wan_dit_sp_begin", "wan_dit_sp_block_qkv",
+           "wan_dit_sp_attention", "wan_dit_sp_block_finish", "wan_dit_sp_end",
+           "wan_vae_create", "wan_vae_load_weights", "wan_vae_missing_weights", "wan_vae_decode", "wan_vae_sync",
+           "wan_vae_last_error", "wan_vae_destroy", "wan_op_conv3d"]
 
 
 class WanError(RuntimeError):
@@ -52,7 +58,10 @@ class wan_dit_config(C.Structure):
 class wan_epilogue(C.Structure):
     _fields_ = [("bias", C.c_void_p), ("out", C.c_void_p), ("ldo", C.c_int64), ("gate0", C.c_void_p),
                 ("gate1", C.c_void_p), ("mod_div", C.c_int), ("mod_ld", C.c_int64),
-                ("up_C", C.c_int), ("up_F", C.c_int), ("up_Hz", C.c_int), ("up_Wz", C.c_int)]
+                ("up_C", C.c_int), ("up_F", C.c_int), ("up_Hz", C.c_int), ("up_Wz", C.c_int),
+                ("gain", C.c_void_p), ("ssq", C.c_void_p), ("ssq_ld", C.c_int64), ("norm_cols", C.c_int),
+                ("rope", C.c_int), ("rope_F", C.c_int), ("rope_H", C.c_int), ("rope_W", C.c_int),
+                ("rope_t", C.c_int), ("rope_h", C.c_int), ("rope_w", C.c_int), ("rope_theta", C.c_float)]
 
 
 _lib = None
@@ -98,6 +107,24 @@ def lib() -> C.CDLL:
         "wan_op_wait_selftest": (I, [I64, P]),
         "wan_op_causal_conv3d": (I, [P, P, I, I, I, I, I, I, P, I64, P, I, I, I, I, P, I64, P, P]),
         "wan_op_set_wait_limit_ns": (None, [I64]),
+        "wan_dit_forward_cfg_euler": (I, [P, P, I, I, I, F, P, I, F, F, F, P, I, P]),
+        "wan_flow_sigmas": (I, [I, D, C.POINTER(D)]),
+        "wan_op_attention_qnorm": (I, [P, I64, P, I64, P, I64, P, I64, I, I, I, I, P, I64, I, F, P]),
+        "wan_op_rms_apply": (I, [P, I64, I, I, P, I64, I, F, P]),
+        "wan_dit_sp_begin": (I, [P, P, I, I, I, I, I, P, I, P, I, I, I, I, P]),
+        "wan_dit_sp_block_qkv": (I, [P, I, P, P]),
+        "wan_dit_sp_attention": (I, [P, P, P, P]),
+        "wan_dit_sp_block_finish": (I, [P, I, P, P]),
+        "wan_dit_sp_end": (I, [P, P, I, P]),
+        "wan_vae_create": (I, [I, I, I, I, C.POINTER(P)]),
+        "wan_vae_load_weights": (I, [P, I, C.POINTER(C.c_char_p), C.POINTER(P), C.POINTER(I),
+                                     C.POINTER(C.POINTER(I64)), C.POINTER(I), I, P]),
+        "wan_vae_missing_weights": (I, [P, C.c_char_p, I]),
+        "wan_vae_decode": (I, [P, P, I, I, I, I, P, I, P]),
+        "wan_vae_sync": (I, [P, P]),
+        "wan_vae_last_error": (C.c_char_p, [P]),
+        "wan_vae_destroy": (None, [P]),
+        "wan_op_conv3d": (I, [P, P, I, I, I, I, I, I, P, I64, P, I, I, I, I, I, P, I64, P, I64, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -227,6 +254,23 @@ class WanDiT:
             self.sync(stream)
         return velocity
 
+    def forward_cfg_euler(self, x, timestep: float, context, guidance: float, sigma: float, sigma_next: float,
+                          x_next=None, stream=None, sync=False):
+        """One fused sampler step of the CFG pair: x f32 [1,C,F,Hz,Wz], context bf16
+        [2,Lc,text_dim] (conditional, unconditional).  Returns x_next (new tensor unless
+        given; may be x itself).  CUDA tensors for device I/O, CPU tensors for host I/O."""
+        import torch
+        _, Cin, F, Hz, Wz = x.shape
+        on_dev = x.is_cuda
+        if x_next is None:
+            x_next = torch.empty(x.shape, dtype=torch.float32, device=x.device, pin_memory=not on_dev)
+        self._check(lib().wan_dit_forward_cfg_euler(self._h, _ptr(x), F, Hz, Wz, float(timestep), _ptr(context),
+                                                    context.shape[1], float(guidance), float(sigma),
+                                                    float(sigma_next), _ptr(x_next), int(on_dev), _stream(stream)))
+        if sync:
+            self.sync(stream)
+        return x_next
+
     def sync(self, stream=None):
         self._check(lib().wan_dit_sync(self._h, _stream(stream)))
 
@@ -247,6 +291,91 @@ class WanDiT:
 
     def flops(self, B, F, Hz, Wz, Lc, per_token=0, Li=0) -> float:
         return lib().wan_dit_flops_image(self._h, B, F, Hz, Wz, Lc, per_token, Li)
+
+
+def flow_sigmas(steps: int, shift: float):
+    """steps + 1 flow-shifted noise levels from 1 down to 0 (wan_flow_sigmas)."""
+    out = (C.c_double * (steps + 1))()
+    _check(lib().wan_flow_sigmas(int(steps), float(shift), out), "wan_flow_sigmas")
+    return list(out)
+
+
+def _weight_arrays(weights):
+    """ctypes arrays of names, pointers, dtypes and shapes of a name -> tensor dict."""
+    items = list(weights.items())
+    on_dev = items[0][1].is_cuda
+    keep = [t.contiguous() for _, t in items]
+    if any(t.is_cuda != on_dev for t in keep):
+        raise ValueError("all tensors of one load call must be on the same side (host or device)")
+    n = len(items)
+    names = (C.c_char_p * n)(*[k.encode() for k, _ in items])
+    ptrs = (C.c_void_p * n)(*[t.data_ptr() for t in keep])
+    dts = (C.c_int * n)(*[_dtype_code(t) for t in keep])
+    shape_arrs = [(C.c_int64 * max(1, t.dim()))(*t.shape) for t in keep]
+    shapes = (C.POINTER(C.c_int64) * n)(*[C.cast(a, C.POINTER(C.c_int64)) for a in shape_arrs])
+    nd = (C.c_int * n)(*[t.dim() for t in keep])
+    return n, names, ptrs, dts, shapes, nd, on_dev, (keep, shape_arrs)
+
+
+class WanVAE:
+    """Handle of ``wan_vae`` (include/wanvae.h): the Wan2.1 VAE decoder."""
+
+    def __init__(self, max_batch: int, max_h: int, max_w: int, device: int = 0):
+        self._h = C.c_void_p()
+        _check(lib().wan_vae_create(int(device), int(max_batch), int(max_h), int(max_w), C.byref(self._h)),
+               "wan_vae_create")
+
+    def close(self):
+        if self._h:
+            lib().wan_vae_destroy(self._h)
+            self._h = C.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, status):
+        if status != 0:
+            raise WanError(status, lib().wan_vae_last_error(self._h).decode())
+
+    def load_weights(self, weights: Dict[str, "object"], stream=None):
+        if not weights:
+            return
+        n, names, ptrs, dts, shapes, nd, on_dev, _keep = _weight_arrays(weights)
+        self._check(lib().wan_vae_load_weights(self._h, n, names, ptrs, dts, shapes, nd, int(on_dev),
+                                               _stream(stream) if on_dev else None))
+
+    def missing_weights(self):
+        buf = C.create_string_buffer(1 << 16)
+        n = lib().wan_vae_missing_weights(self._h, buf, len(buf))
+        return n, buf.value.decode()
+
+    def decode(self, z, video=None, stream=None, sync=False):
+        """z f32 [B, 16, T, H, W] (CUDA or CPU) -> video f32 [B, 3, 1 + 4 (T - 1), 8 H, 8 W]."""
+        import torch
+        B, _, T, H, W = z.shape
+        on_dev = z.is_cuda
+        if video is None:
+            video = torch.empty(B, 3, 1 + 4 * (T - 1), 8 * H, 8 * W, dtype=torch.float32, device=z.device,
+                                pin_memory=not on_dev)
+        self._check(lib().wan_vae_decode(self._h, _ptr(z), B, T, H, W, _ptr(video), int(on_dev), _stream(stream)))
+        if sync:
+            self._check(lib().wan_vae_sync(self._h, _stream(stream)))
+        return video
+
+
+def op_conv3d(x, w_packed, bias, y, kernel, Co, cache=None, add=None, time_split=False, stream=None):
+    """Implicit-GEMM causal Conv3d: x bf16 [B,T,H,W,Ci] (channels last), w_packed bf16
+    [Co_pad, ldw] ((kt,kh,kw,ci) order, ci padded to a multiple of 64), y bf16 rows with
+    channel stride y.shape[-1], cache [B,nc,H,W,Ci] or None, add residual or None."""
+    B, T, H, W, Ci = x.shape
+    kt, kh, kw = kernel
+    nc = 0 if cache is None else cache.shape[1]
+    _check(lib().wan_op_conv3d(_ptr(x), _ptr(cache), nc, B, T, H, W, Ci, _ptr(w_packed), w_packed.stride(0),
+                               _ptr(bias), Co, w_packed.shape[0], kt, kh, kw, _ptr(y), y.shape[-1], _ptr(add),
+                               0 if add is None else add.shape[-1], int(time_split), _stream(stream)), "wan_op_conv3d")
 
 
 def moe_select(t: float, boundary: float, num_train_timesteps: int = 1000) -> int:
@@ -277,12 +406,17 @@ class WanMoE:
 
 # ---------------------------------------------------------------- op-level wrappers
 def op_gemm(A, W, epilogue: str, out, bias=None, gate0=None, gate1=None, mod_div=1, mod_ld=0,
-            unpatch=(0, 0, 0, 0), M=None, stream=None):
+            unpatch=(0, 0, 0, 0), M=None, stream=None, gain=None, ssq=None, norm_cols=0, rope_grid=None,
+            rope_split=(44, 42, 42), rope_theta=10000.0):
     M = A.shape[0] if M is None else M
     N, K = W.shape
+    rg = rope_grid or (0, 0, 0)
     e = wan_epilogue(bias=_ptr(bias), out=_ptr(out), ldo=(out.stride(0) if out.dim() == 2 else 0),
                      gate0=_ptr(gate0), gate1=_ptr(gate1), mod_div=mod_div, mod_ld=mod_ld,
-                     up_C=unpatch[0], up_F=unpatch[1], up_Hz=unpatch[2], up_Wz=unpatch[3])
+                     up_C=unpatch[0], up_F=unpatch[1], up_Hz=unpatch[2], up_Wz=unpatch[3],
+                     gain=_ptr(gain), ssq=_ptr(ssq), ssq_ld=(ssq.stride(0) if ssq is not None else 0),
+                     norm_cols=norm_cols, rope=int(rope_grid is not None), rope_F=rg[0], rope_H=rg[1], rope_W=rg[2],
+                     rope_t=rope_split[0], rope_h=rope_split[1], rope_w=rope_split[2], rope_theta=rope_theta)
     _check(lib().wan_op_gemm(_ptr(A), A.stride(0), _ptr(W), W.stride(0), M, N, K, EPI[epilogue], C.byref(e),
                              _stream(stream)), "wan_op_gemm")
 
@@ -304,6 +438,18 @@ def op_attention(q, k, v, o, B, heads, Lq, Lk, ldq=None, ldk=None, ldv=None, ldo
     _check(lib().wan_op_attention(_ptr(q), ldq or q.stride(0), _ptr(k), ldk or k.stride(0), _ptr(v),
                                   ldv or v.stride(0), _ptr(o), ldo or o.stride(0), B, heads, Lq, Lk,
                                   _stream(stream)), "wan_op_attention")
+
+
+def op_attention_qnorm(q_ptr, ldq, k_ptr, ldk, v_ptr, ldv, o, B, heads, Lq, Lk, q_ssq, ngroups, eps, stream=None):
+    """Attention with unnormalised queries scaled by their RMSNorm row factors."""
+    _check(lib().wan_op_attention_qnorm(q_ptr, ldq, k_ptr, ldk, v_ptr, ldv, _ptr(o), o.stride(0), B, heads, Lq, Lk,
+                                        _ptr(q_ssq), q_ssq.stride(0), ngroups, eps, _stream(stream)),
+           "wan_op_attention_qnorm")
+
+
+def op_rms_apply(buf_ptr, ld, rows, D, ssq_ptr, ssq_ld, ngroups, eps, stream=None):
+    _check(lib().wan_op_rms_apply(buf_ptr, ld, rows, D, ssq_ptr, ssq_ld, ngroups, eps, _stream(stream)),
+           "wan_op_rms_apply")
 
 
 def op_attention_ptr(q, ldq, k, ldk, v, ldv, o, ldo, B, heads, Lq, Lk, stream=None):

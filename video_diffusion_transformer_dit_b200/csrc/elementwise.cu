@@ -160,14 +160,6 @@ cudaError_t launch_mod_combine(const float* sst, const float* tproj, float* out,
 }
 
 // ------------------------------------------------------------------ RMSNorm across heads + RoPE
-// Pair p (0..63) of a 128-wide head: axis t for p < nt, h for p < nt + nh, else w.
-__device__ __forceinline__ float2 rope_cs(const RopeTables& rt, int p, int f, int i, int j) {
-    if (p < rt.nt) return __ldg(rt.t + f * rt.nt + p);
-    p -= rt.nt;
-    if (p < rt.nh) return __ldg(rt.h + i * rt.nh + p);
-    p -= rt.nh;
-    return __ldg(rt.w + j * rt.nw + p);
-}
 
 template <int NCH>
 __global__ void __launch_bounds__(256) rmsnorm_rope_kernel(__nv_bfloat16* buf, long long ld, int rows, float eps,
@@ -347,25 +339,146 @@ cudaError_t launch_rmsnorm_rope(void* buf, long long ld, int rows, int D, float 
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ RMSNorm row factor applied in place
+// The sums of squares come from the q/k projection's epilogue; one warp per
+// row, the row factor from the row's group sums (fixed order), 16-byte
+// vectors, every load of the row issued before any store.
+template <int NCH>
+__global__ void __launch_bounds__(256) rms_apply_kernel(__nv_bfloat16* buf, long long ld, int rows, RowNorm rn) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= rows) return;
+    __nv_bfloat16* xr = buf + (long long)row * ld;
+    uint4 u[NCH];
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) u[t] = *reinterpret_cast<const uint4*>(xr + (t * 32 + lane) * 8);
+    const float* g = rn.ssq + (long long)row * rn.ssq_ld;
+    float ss = 0.f;
+    for (int k = 0; k < rn.ngroups; ++k) ss += __ldg(g + k);
+    const float sc = rsqrtf(ss * rn.inv_n + rn.eps);
+    const uint64_t sc2 = f2pack(sc, sc);
+#pragma unroll
+    for (int t = 0; t < NCH; ++t) {
+        const uint32_t w[4] = {u[t].x, u[t].y, u[t].z, u[t].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const float2 f = unpack_bf16(w[h]);
+            float a, b;
+            f2unpack(mul2(f2pack(f.x, f.y), sc2), a, b);
+            o[h] = pack_bf16(a, b);
+        }
+        *reinterpret_cast<uint4*>(xr + (t * 32 + lane) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+cudaError_t launch_rms_apply(void* buf, long long ld, int rows, int D, const RowNorm& rn, const LaunchCtx& ctx) {
+    if (rows <= 0) return cudaSuccess;
+    if (!rn.ssq || rn.ngroups <= 0 || !rmsnorm_rope_shape_ok(D, ld) ||
+        (reinterpret_cast<uintptr_t>(buf) & 15))
+        return cudaErrorInvalidValue;
+    auto Bp = reinterpret_cast<__nv_bfloat16*>(buf);
+    const int grid = (rows + 7) / 8;
+#define WAN_RMS_APPLY_CASE(n)                                                             \
+    case n:                                                                               \
+        rms_apply_kernel<n><<<grid, 256, 0, ctx.stream>>>(Bp, ld, rows, rn);              \
+        break;
+    switch (D / 256) {
+        WAN_RMS_APPLY_CASE(1) WAN_RMS_APPLY_CASE(2) WAN_RMS_APPLY_CASE(3) WAN_RMS_APPLY_CASE(4)
+        WAN_RMS_APPLY_CASE(6) WAN_RMS_APPLY_CASE(8) WAN_RMS_APPLY_CASE(12) WAN_RMS_APPLY_CASE(16)
+        WAN_RMS_APPLY_CASE(20) WAN_RMS_APPLY_CASE(24)
+        default: return cudaErrorInvalidValue;
+    }
+#undef WAN_RMS_APPLY_CASE
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ sequence-parallel exchange layouts
+// pack:   send[((b * P + j) * Ls + l) * 3hd + s * hd + c] = qkv[(b * Ls + l) * 3D + s * D + j * hd + c]
+// unpack: o[(b * Ls + l) * D + j * hd + c]               = back[((b * P + j) * Ls + l) * hd + c]
+// (s = q, k, v; hd = 128 * heads / P columns of head group j); 8 bf16 per thread step.
+__global__ void sp_pack_kernel(const __nv_bfloat16* __restrict__ qkv, __nv_bfloat16* __restrict__ send, int B, int P,
+                               int Ls, int D, int hd) {
+    const int v8 = 3 * hd / 8;  // 16-byte vectors per packed row
+    const long long total = (long long)B * P * Ls * v8;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int c8 = idx % v8;
+        const long long rest = idx / v8;
+        const int l = rest % Ls;
+        const long long bj = rest / Ls;
+        const int j = bj % P;
+        const int b = bj / P;
+        const int sidx = c8 / (hd / 8), cc = (c8 % (hd / 8)) * 8;
+        const uint4 v = *reinterpret_cast<const uint4*>(qkv + ((long long)b * Ls + l) * 3 * D + (long long)sidx * D +
+                                                        (long long)j * hd + cc);
+        *reinterpret_cast<uint4*>(send + idx * 8) = v;
+    }
+}
+
+__global__ void sp_unpack_kernel(const __nv_bfloat16* __restrict__ back, __nv_bfloat16* __restrict__ o, int B, int P,
+                                 int Ls, int D, int hd) {
+    const int v8 = hd / 8;
+    const long long total = (long long)B * P * Ls * v8;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int c8 = idx % v8;
+        const long long rest = idx / v8;
+        const int l = rest % Ls;
+        const long long bj = rest / Ls;
+        const int j = bj % P;
+        const int b = bj / P;
+        const uint4 v = *reinterpret_cast<const uint4*>(back + idx * 8);
+        *reinterpret_cast<uint4*>(o + ((long long)b * Ls + l) * D + (long long)j * hd + c8 * 8) = v;
+    }
+}
+
+cudaError_t launch_sp_pack(const void* qkv, void* send, int B, int P, int Ls, int D, const LaunchCtx& ctx) {
+    if (B <= 0 || Ls <= 0) return cudaSuccess;
+    if (P <= 0 || D % P || (D / P) % 8 || ((reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(send)) & 15))
+        return cudaErrorInvalidValue;
+    const long long total = (long long)B * Ls * 3 * D / 8;
+    long long g = (total + 255) / 256;
+    if (g > ctx.num_sms * 16) g = ctx.num_sms * 16;
+    sp_pack_kernel<<<(int)g, 256, 0, ctx.stream>>>(reinterpret_cast<const __nv_bfloat16*>(qkv),
+                                                  reinterpret_cast<__nv_bfloat16*>(send), B, P, Ls, D, D / P);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sp_unpack(const void* back, void* o, int B, int P, int Ls, int D, const LaunchCtx& ctx) {
+    if (B <= 0 || Ls <= 0) return cudaSuccess;
+    if (P <= 0 || D % P || (D / P) % 8 || ((reinterpret_cast<uintptr_t>(back) | reinterpret_cast<uintptr_t>(o)) & 15))
+        return cudaErrorInvalidValue;
+    const long long total = (long long)B * Ls * D / 8;
+    long long g = (total + 255) / 256;
+    if (g > ctx.num_sms * 16) g = ctx.num_sms * 16;
+    sp_unpack_kernel<<<(int)g, 256, 0, ctx.stream>>>(reinterpret_cast<const __nv_bfloat16*>(back),
+                                                    reinterpret_cast<__nv_bfloat16*>(o), B, P, Ls, D, D / P);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ patchify / unpatchify
 // X[b * L + (f * Hp + i) * Wp + j, c * 4 + kh * 2 + kw] = latent[b, c, f, 2i + kh, 2j + kw]
 // for c < C; columns [4C, ldx) of every row are written as zeros (K padding of
 // the patch GEMM when 4C is not a multiple of its K tile).
 template <typename T>
 __global__ void patchify_kernel(const T* __restrict__ lat, __nv_bfloat16* __restrict__ X, int B, int C, int F, int Hz,
-                                int Wz, int ldx) {
+                                int Wz, int ldx, int tok0, int rows) {
     const int Hp = Hz >> 1, Wp = Wz >> 1;
     const long long L = (long long)F * Hp * Wp;
     const int G = ldx >> 2;  // groups of 4 columns per row
-    const long long total = (long long)B * L * G;
+    const long long total = (long long)B * rows * G;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
         const int c = idx % G;
         const long long row = idx / G;
         uint2 u = make_uint2(0u, 0u);
-        if (c < C) {
-            const int b = row / L;
-            const long long l = row - (long long)b * L;
+        const int b = row / rows;
+        const long long l = tok0 + (row - (long long)b * rows);
+        if (c < C && l < L) {
             const int f = l / (Hp * Wp);
             const int rem = l - (long long)f * (Hp * Wp);
             const int i = rem / Wp, j = rem - (rem / Wp) * Wp;
@@ -378,20 +491,24 @@ __global__ void patchify_kernel(const T* __restrict__ lat, __nv_bfloat16* __rest
 }
 
 cudaError_t launch_patchify(const void* latent, int latent_dtype, int B, int C, int F, int Hz, int Wz, void* X,
-                            int ldx, const LaunchCtx& ctx) {
-    if (ldx < 4 * C || ldx % 4) return cudaErrorInvalidValue;
-    const long long total = (long long)B * F * (Hz / 2) * (Wz / 2) * (ldx / 4);
+                            int ldx, const LaunchCtx& ctx, int tok0, int rows) {
+    if (ldx < 4 * C || ldx % 4 || tok0 < 0 || rows < 0) return cudaErrorInvalidValue;
+    if (rows == 0) {
+        rows = F * (Hz / 2) * (Wz / 2);
+        tok0 = 0;
+    }
+    const long long total = (long long)B * rows * (ldx / 4);
     if (total <= 0) return cudaSuccess;
     int grid = (int)((total + 255) / 256);
     if (grid > ctx.num_sms * 16) grid = ctx.num_sms * 16;
     if (latent_dtype == 0)
         patchify_kernel<float><<<grid, 256, 0, ctx.stream>>>(reinterpret_cast<const float*>(latent),
                                                               reinterpret_cast<__nv_bfloat16*>(X), B, C, F, Hz, Wz,
-                                                              ldx);
+                                                              ldx, tok0, rows);
     else
         patchify_kernel<__nv_bfloat16><<<grid, 256, 0, ctx.stream>>>(reinterpret_cast<const __nv_bfloat16*>(latent),
                                                                       reinterpret_cast<__nv_bfloat16*>(X), B, C, F, Hz,
-                                                                      Wz, ldx);
+                                                                      Wz, ldx, tok0, rows);
     if (ctx.launches) ++*ctx.launches;
     return cudaGetLastError();
 }
@@ -617,16 +734,17 @@ __global__ void cfg_euler_kernel(const float* __restrict__ x, const float* __res
         const float4 a = reinterpret_cast<const float4*>(x)[i];
         const float4 c = reinterpret_cast<const float4*>(vc)[i];
         float4 v = c;
-        if (vu) {
+        if (vu) {  // fused multiply-adds spelled out: the proj_out epilogue computes the same roundings
             const float4 u = reinterpret_cast<const float4*>(vu)[i];
-            v = make_float4(u.x + s * (c.x - u.x), u.y + s * (c.y - u.y), u.z + s * (c.z - u.z), u.w + s * (c.w - u.w));
+            v = make_float4(__fmaf_rn(s, c.x - u.x, u.x), __fmaf_rn(s, c.y - u.y, u.y), __fmaf_rn(s, c.z - u.z, u.z),
+                            __fmaf_rn(s, c.w - u.w, u.w));
         }
-        reinterpret_cast<float4*>(xn)[i] =
-            make_float4(a.x + dsigma * v.x, a.y + dsigma * v.y, a.z + dsigma * v.z, a.w + dsigma * v.w);
+        reinterpret_cast<float4*>(xn)[i] = make_float4(__fmaf_rn(dsigma, v.x, a.x), __fmaf_rn(dsigma, v.y, a.y),
+                                                       __fmaf_rn(dsigma, v.z, a.z), __fmaf_rn(dsigma, v.w, a.w));
     }
     for (long long i = n4 * 4 + blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += stride) {
-        const float v = vu ? vu[i] + s * (vc[i] - vu[i]) : vc[i];
-        xn[i] = x[i] + dsigma * v;
+        const float v = vu ? __fmaf_rn(s, vc[i] - vu[i], vu[i]) : vc[i];
+        xn[i] = __fmaf_rn(dsigma, v, x[i]);
     }
 }
 
@@ -640,6 +758,26 @@ cudaError_t launch_cfg_euler(const float* x, const float* v_cond, const float* v
     if (g < 1) g = 1;
     if (g > ctx.num_sms * 8) g = ctx.num_sms * 8;
     cfg_euler_kernel<<<(int)g, 256, 0, ctx.stream>>>(x, v_cond, v_uncond, guidance, sigma_next - sigma, n, x_next);
+    if (ctx.launches) ++*ctx.launches;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ per-call sampler scalars
+// sched = {guidance, sigma_next - sigma}; t[0..nt) = t_value.  Kernel arguments
+// carry the values, so a captured forward reads them from device memory.
+__global__ void set_sampler_scalars_kernel(float* sched, float guidance, float dsigma, float* t, int nt,
+                                           float t_value) {
+    const int i = threadIdx.x;
+    if (i == 0) {
+        sched[0] = guidance;
+        sched[1] = dsigma;
+    }
+    for (int k = i; k < nt; k += blockDim.x) t[k] = t_value;
+}
+
+cudaError_t launch_set_sampler_scalars(float* sched, float guidance, float dsigma, float* t, int nt, float t_value,
+                                       const LaunchCtx& ctx) {
+    set_sampler_scalars_kernel<<<1, 32, 0, ctx.stream>>>(sched, guidance, dsigma, t, nt, t_value);
     if (ctx.launches) ++*ctx.launches;
     return cudaGetLastError();
 }

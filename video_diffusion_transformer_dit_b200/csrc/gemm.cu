@@ -30,15 +30,18 @@ struct GemmParams {
     WaitCtl wc;
 };
 
-template <int BN>
+// PAIR: two A tiles per stage (rows r and r + pair_off) against one W tile,
+// two accumulators per tile (the CFG pair of EPI_CFG_EULER).
+template <int BN, bool PAIR = false>
 struct GemmCfg {
     static constexpr int BM = 128;
     static constexpr int BK = 64;
+    static constexpr int NA = PAIR ? 2 : 1;
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = BN * BK * 2;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
     static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
-    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int TMEM_COLS = 2 * NA * BN;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 };
 
@@ -247,10 +250,12 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
             break;
         }
         case EPI_UNPATCHIFY: {
-            // row = b * L + token, token = (f * Hp + i) * Wp + j; column = (kh * 2 + kw) * C + ch
+            // row = b * rows + r, token l = tok0 + r = (f * Hp + i) * Wp + j; column = (kh * 2 + kw) * C + ch
             const int Hp = e.Hz >> 1, Wp = e.Wz >> 1;
-            const int b = row / e.L;
-            const int l = row - b * e.L;
+            const int rows = e.up_rows > 0 ? e.up_rows : e.L;
+            const int b = row / rows;
+            const int l = e.up_tok0 + (row - b * rows);
+            if (l >= e.L) break;  // a padding row of a sequence shard
             const int f = l / (Hp * Wp);
             const int rem = l - f * (Hp * Wp);
             const int ii = rem / Wp;
@@ -274,6 +279,94 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
     }
 }
 
+// EPI_QK_NORM on 32 consecutive columns [c, c + 32) of one row.  For normed
+// columns the sum of squares of acc + bias is returned (fp32, before the
+// gain) and the stored value is gain * (acc + bias), rotated pair by pair
+// ((x0, x1) -> (x0 cos - x1 sin, x1 cos + x0 sin)) when RoPE is on; the row
+// factor rsqrt(mean + eps) commutes with both and is applied later.  All of
+// it on packed fp32 pairs, so the scalar FP32 pipe stays free for MMA issue.
+__device__ __forceinline__ float epilogue_qk_chunk(const EpiParams& e, int row, int c, const uint32_t (&r)[32],
+                                                   bool normed, int f, int ii, int jj) {
+    uint64_t v2[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v2[i] = f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+    if (e.bias) {
+        const ulonglong2* b2 = reinterpret_cast<const ulonglong2*>(e.bias + c);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const ulonglong2 b = __ldg(b2 + i);
+            v2[2 * i] = add2(v2[2 * i], b.x);
+            v2[2 * i + 1] = add2(v2[2 * i + 1], b.y);
+        }
+    }
+    float ss = 0.0f;
+    if (normed) {
+        uint64_t s2 = 0ull;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s2 = fma2(v2[i], v2[i], s2);
+        float sa, sb;
+        f2unpack(s2, sa, sb);
+        ss = sa + sb;
+        const ulonglong2* g2 = reinterpret_cast<const ulonglong2*>(e.gain + c);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const ulonglong2 g = __ldg(g2 + i);
+            v2[2 * i] = mul2(v2[2 * i], g.x);
+            v2[2 * i + 1] = mul2(v2[2 * i + 1], g.y);
+        }
+        if (e.rope.t) {
+            const int p0 = (c & 127) >> 1;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float2 cs = rope_cs(e.rope, p0 + i, f, ii, jj);
+                float a, b;
+                f2unpack(v2[i], a, b);
+                v2[i] = fma2(v2[i], f2pack(cs.x, cs.x), mul2(f2pack(b, a), f2pack(-cs.y, cs.y)));
+            }
+        }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            float a, b;
+            f2unpack(v2[4 * i + h], a, b);
+            w[h] = pack_bf16(a, b);
+        }
+        dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return ss;
+}
+
+// CFG + Euler on 32 consecutive columns [c, c + 32) of one token row: both
+// velocities rounded to bf16 as proj_out's output is, then
+// x_next = x + dsigma * (v_u + s (v_c - v_u)) at the unpatchify position.
+__device__ __forceinline__ void epilogue_cfg_euler(const EpiParams& e, int row, int c, const uint32_t (&rc)[32],
+                                                   const uint32_t (&ru)[32]) {
+    const float s = __ldg(e.sched), dsig = __ldg(e.sched + 1);
+    const int Hp = e.Hz >> 1, Wp = e.Wz >> 1;
+    const int f = row / (Hp * Wp);
+    const int rem = row - f * (Hp * Wp);
+    const int ii = rem / Wp;
+    const int jj = rem - ii * Wp;
+    float* xn = reinterpret_cast<float*>(e.out);
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+        const int col = c + t;
+        const int ch = col % e.C;
+        const int sub = col / e.C;
+        const int kh = sub >> 1, kw = sub & 1;
+        const long long idx = (((long long)ch * e.F + f) * e.Hz + (2 * ii + kh)) * e.Wz + (2 * jj + kw);
+        const float bias = e.bias ? __ldg(e.bias + col) : 0.0f;
+        const float vc = __bfloat162float(__float2bfloat16_rn(__uint_as_float(rc[t]) + bias));
+        const float vu = __bfloat162float(__float2bfloat16_rn(__uint_as_float(ru[t]) + bias));
+        const float v = __fmaf_rn(s, vc - vu, vu);
+        xn[idx] = __fmaf_rn(dsig, v, __ldg(e.x + idx));
+    }
+}
+
 constexpr int EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
 
@@ -281,12 +374,13 @@ template <int BN, int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
-    using Cfg = GemmCfg<BN>;
+    constexpr bool PAIR = KIND == EPI_CFG_EULER;
+    using Cfg = GemmCfg<BN, PAIR>;
     constexpr int STAGES = Cfg::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+    uint8_t* sA = smem;                                   // [STAGES][NA] A tiles
+    uint8_t* sB = smem + STAGES * Cfg::NA * Cfg::A_BYTES;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
@@ -342,7 +436,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         break;
                     }
                     mbar_expect_tx(full + stage, Cfg::STAGE_BYTES);
-                    tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, full + stage, kb * Cfg::BK, mb * Cfg::BM);
+                    tma_load_2d(sA + stage * Cfg::NA * Cfg::A_BYTES, &tmA, full + stage, kb * Cfg::BK, mb * Cfg::BM);
+                    if constexpr (PAIR)
+                        tma_load_2d(sA + (stage * 2 + 1) * Cfg::A_BYTES, &tmA, full + stage, kb * Cfg::BK,
+                                    p.epi.pair_off + mb * Cfg::BM);
                     tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, full + stage, kb * Cfg::BK, nb * BN);
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -357,6 +454,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
             constexpr uint32_t IDESC = idesc_bf16(128, BN, false);
+            constexpr int ACC_COLS = Cfg::NA * BN;            // TMEM columns of one accumulator set
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -368,19 +466,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * BN;
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(full + stage, phase, abort_flag, p.wc)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * Cfg::A_BYTES);
+                    const uint32_t a0 = smem_u32(sA + stage * Cfg::NA * Cfg::A_BYTES);
                     const uint32_t b0 = smem_u32(sB + stage * Cfg::B_BYTES);
 #pragma unroll
                     for (int k = 0; k < Cfg::BK / 16; ++k) {
                         umma_bf16_ss(d_tmem, sdesc_kmajor_sw128(a0 + 32 * k), sdesc_kmajor_sw128(b0 + 32 * k), IDESC,
                                      (kb | k) != 0);
+                        if constexpr (PAIR)
+                            umma_bf16_ss(d_tmem + BN, sdesc_kmajor_sw128(a0 + Cfg::A_BYTES + 32 * k),
+                                         sdesc_kmajor_sw128(b0 + 32 * k), IDESC, (kb | k) != 0);
                     }
                     issued = true;
                     umma_commit(empty + stage);
@@ -409,13 +510,44 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc))) break;
             tc_fence_after();
             const int row = mb * 128 + q * 32 + lane;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * (Cfg::NA * BN);
+            if constexpr (KIND == EPI_QK_NORM) {
+                // this warp's 128 columns are one head: its sum of squares is one ssq entry
+                static_assert(BN == 256, "one 128-column group per epilogue warp");
+                const int gcol = nb * BN + chalf * CW;
+                const bool normed = gcol < p.epi.norm_cols;
+                int f = 0, ii = 0, jj = 0;
+                if (normed && p.epi.rope.t) {
+                    const int hw = p.epi.rope.Hp * p.epi.rope.Wp;
+                    const int l = min(p.epi.rope_tok0 + row % p.epi.rope_L, p.epi.rope.Fp * hw - 1);
+                    f = l / hw;
+                    const int rem = l - f * hw;
+                    ii = rem / p.epi.rope.Wp;
+                    jj = rem - ii * p.epi.rope.Wp;
+                }
+                float ss = 0.0f;
+#pragma unroll 1
+                for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(taddr + c0, r);
+                    tmem_ld_wait(r);
+                    if (row < p.M) ss += epilogue_qk_chunk(p.epi, row, nb * BN + c0, r, normed, f, ii, jj);
+                }
+                if (normed && row < p.M) p.epi.ssq[(long long)row * p.epi.ssq_ld + gcol / 128] = ss;
+            } else
 #pragma unroll 1
             for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
                 uint32_t r[32];
                 tmem_ld32(taddr + c0, r);
                 tmem_ld_wait(r);
-                if (row < p.M) epilogue_chunk<KIND>(p.epi, row, nb * BN + c0, r);
+                if constexpr (PAIR) {
+                    uint32_t ru[32];
+                    tmem_ld32(taddr + BN + c0, ru);
+                    tmem_ld_wait(ru);
+                    if (row < p.M) epilogue_cfg_euler(p.epi, row, nb * BN + c0, r, ru);
+                } else {
+                    if (row < p.M) epilogue_chunk<KIND>(p.epi, row, nb * BN + c0, r);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -447,7 +579,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 template <int BN, int KIND>
 static cudaError_t set_gemm_attr_one() {
     return cudaFuncSetAttribute(gemm_tc_kernel<BN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                GemmCfg<BN>::SMEM_BYTES);
+                                GemmCfg<BN, KIND == EPI_CFG_EULER>::SMEM_BYTES);
 }
 
 template <int BN>
@@ -466,6 +598,8 @@ cudaError_t init_gemm_attributes() {
     cudaError_t e = set_gemm_attr<256>();
     if (e == cudaSuccess) e = set_gemm_attr<128>();
     if (e == cudaSuccess) e = set_gemm_attr<64>();
+    if (e == cudaSuccess) e = set_gemm_attr_one<64, EPI_CFG_EULER>();
+    if (e == cudaSuccess) e = set_gemm_attr_one<256, EPI_QK_NORM>();
     return e;
 }
 
@@ -474,6 +608,18 @@ static cudaError_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, 
                                   const LaunchCtx& ctx) {
     using Cfg = GemmCfg<BN>;
     const int grid = p.num_tiles < ctx.num_sms ? p.num_tiles : ctx.num_sms;
+    if (p.epi.kind == EPI_CFG_EULER) {  // 64-column tiles only (proj_out: N = 4 * out_ch)
+        if (BN != 64) return cudaErrorInvalidValue;
+        gemm_tc_kernel<64, EPI_CFG_EULER><<<grid, GEMM_THREADS, GemmCfg<64, true>::SMEM_BYTES, ctx.stream>>>(ta, tb, p);
+        if (ctx.launches) ++*ctx.launches;
+        return cudaGetLastError();
+    }
+    if (p.epi.kind == EPI_QK_NORM) {  // 256-column tiles only: one head per epilogue warp
+        if (BN != 256) return cudaErrorInvalidValue;
+        gemm_tc_kernel<256, EPI_QK_NORM><<<grid, GEMM_THREADS, GemmCfg<256>::SMEM_BYTES, ctx.stream>>>(ta, tb, p);
+        if (ctx.launches) ++*ctx.launches;
+        return cudaGetLastError();
+    }
     switch (p.epi.kind) {
 #define WAN_GEMM_CASE(K)                                                                   \
     case K:                                                                                \
@@ -501,6 +647,17 @@ cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long l
         return cudaErrorInvalidValue;
     if ((reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(W) & 15)) return cudaErrorInvalidValue;
     int BN = (N % 256 == 0) ? 256 : (N % 128 == 0) ? 128 : 64;
+    const bool pair = epi.kind == EPI_CFG_EULER;
+    if (pair) {
+        BN = 64;
+        if (epi.pair_off < M || !epi.x || !epi.sched || !epi.out) return cudaErrorInvalidValue;
+    }
+    if (epi.kind == EPI_QK_NORM) {
+        if (N % 256 || epi.norm_cols < 0 || epi.norm_cols % 128 || epi.norm_cols > N || !epi.ssq ||
+            (epi.norm_cols > 0 && !epi.gain) || epi.ssq_ld < epi.norm_cols / 128 || epi.ldo % 8 ||
+            (epi.rope.t && epi.rope_L <= 0))
+            return cudaErrorInvalidValue;
+    }
     GemmParams p;
     p.M = M;
     p.N = N;
@@ -515,7 +672,9 @@ cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long l
     p.wc.err = ctx.err;
     p.wc.limit_ns = ctx.wait_limit_ns;
     CUtensorMap ta, tb;
-    if (!make_tmap_2d(&ta, A, K, M, lda, 64, 128)) return cudaErrorInvalidValue;
+    // the pair variant reads the second sample's rows [pair_off, pair_off + M) as well
+    const uint64_t a_rows = pair ? (uint64_t)epi.pair_off + (uint64_t)M : (uint64_t)M;
+    if (!make_tmap_2d(&ta, A, K, a_rows, lda, 64, 128)) return cudaErrorInvalidValue;
     if (!make_tmap_2d(&tb, W, K, N, ldw, 64, BN)) return cudaErrorInvalidValue;
     switch (BN) {
         case 256: return launch_gemm_bn<256>(ta, tb, p, ctx);

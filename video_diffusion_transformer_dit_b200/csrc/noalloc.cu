@@ -104,7 +104,7 @@ extern "C" wan_status wan_op_rmsnorm_rope_noalloc(void* buf, int64_t ld, int row
     fill_rope_table<<<(total + 255) / 256, 256, 0, st>>>(tab, Fp, Hp, Wp, rope_t, rope_h, rope_w,
                                                          std::log((double)theta));
     if (cudaPeekAtLastError() != cudaSuccess) return WAN_ECUDA;
-    RopeTables rt{tab, tab + (size_t)Fp * nt, tab + (size_t)Fp * nt + (size_t)Hp * nh, Fp, Hp, Wp, nt, nh, nw};
+    RopeTables rt{tab, tab + (size_t)Fp * nt, tab + (size_t)Fp * nt + (size_t)Hp * nh, Fp, Hp, Wp, nt, nh, nw, 0};
     cudaError_t e = launch_rmsnorm_rope(buf, ld, rows, D, eps, gain, 0, 1, 0, &rt, Fp * Hp * Wp, ctx);
     return e == cudaSuccess ? WAN_OK : (e == cudaErrorInvalidValue ? WAN_ESHAPE : WAN_ECUDA);
 }

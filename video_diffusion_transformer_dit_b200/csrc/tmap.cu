@@ -54,4 +54,23 @@ bool make_tmap_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t d1, 
     return r == CUDA_SUCCESS;
 }
 
+// 5-D bf16 tensor [d4][d3][d2][d1][inner] (channels-last video: inner = channels,
+// d1 = width, d2 = height, d3 = frames, d4 = batch), strides in elements, box
+// 1 x 1 x box2 x box1 x box_inner; coordinates outside the tensor (negative
+// included) read as zero.
+bool make_tmap_5d(CUtensorMap* m, const void* ptr, const uint64_t (&dims)[5], const uint64_t (&strides_elems)[4],
+                  uint32_t box_inner, uint32_t box1, uint32_t box2) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t d[5], st[4];
+    for (int i = 0; i < 5; ++i) d[i] = dims[i];
+    for (int i = 0; i < 4; ++i) st[i] = strides_elems[i] * 2;
+    cuuint32_t box[5] = {box_inner, box1, box2, 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), d, st, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace wan

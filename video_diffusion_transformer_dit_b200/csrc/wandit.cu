@@ -6,6 +6,7 @@
 // forward is the diffusers WanTransformer3DModel forward (pswp.cn notes on
 // WanPipeline, sections "WanTransformer3DModel" and "WanTransformerBlock")
 // expressed as launches of the sm_100a kernels in this directory.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -18,6 +19,7 @@
 
 #include "../../include/wandit.h"
 #include "../../include/wandit_ops.h"
+#include "../../include/wanvae.h"
 #include "kernels.h"
 
 using wan::EpiParams;
@@ -80,7 +82,7 @@ struct Plan {
     int timed_pairs = 0;        // pairs recorded by the most recent timed forward
 };
 
-using PlanKey = std::tuple<int, int, int, int, int, int, int, int>;
+using PlanKey = std::tuple<int, int, int, int, int, int, int, int, int, int, int, int>;
 
 }  // namespace
 
@@ -114,6 +116,8 @@ struct wan_dit {
     void *img_stage = nullptr, *ih = nullptr, *ictx = nullptr, *kvi = nullptr, *o2 = nullptr;  // image branch
     float *temb, *tproj, *th32;
     float* modc;          // [N, max_batch, 6, D] per-sample modulation of every block
+    float* sched;         // {guidance, sigma_next - sigma} of the fused sampler step
+    float* ssq;           // [R, 3 * heads] per-head sums of squares: self q | self k | cross q
     int* d_err = nullptr;
     // options / state
     bool use_graph = true;
@@ -125,6 +129,12 @@ struct wan_dit {
     bool timing = false;
     Plan* last_plan = nullptr;
     bool last_timed = false;
+    // sequence-parallel forward in progress (between wan_dit_sp_begin and wan_dit_sp_end)
+    bool sp_active = false;
+    int sp_B = 0, sp_F = 0, sp_Hz = 0, sp_Wz = 0, sp_Lc = 0, sp_per_token = 0, sp_dtype = 0;
+    int sp_rank = 0, sp_world = 0, sp_Ls = 0;
+    int sp_next_block = 0;
+    int sp_phase = 0;     // 0: next call is sp_block_qkv, 1: sp_block_finish
 };
 
 namespace {
@@ -142,6 +152,12 @@ wan_status cuda_fail(wan_dit* h, cudaError_t e, const char* what) {
     do {                                            \
         cudaError_t e_ = (call);                    \
         if (e_ != cudaSuccess) return cuda_fail(h, e_, what); \
+    } while (0)
+
+#define WAN_CU_RET(call)                  \
+    do {                                  \
+        wan_status s_ = (call);           \
+        if (s_ != WAN_OK) return s_;      \
     } while (0)
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -326,6 +342,8 @@ wan_status build_workspace(wan_dit* h) {
         {(void**)&h->temb, (size_t)(R * D * 4)},       {(void**)&h->tproj, (size_t)(R * 6 * D * 4)},
         {(void**)&h->th32, (size_t)(R * D * 4)},
         {(void**)&h->modc, (size_t)((long long)N * c.max_batch * 6 * D * 4)},
+        {(void**)&h->sched, (size_t)64},
+        {(void**)&h->ssq, (size_t)(R * 3 * c.heads * 4)},
     };
     if (Ri > 0) {
         items.push_back({&h->img_stage, (size_t)(Ri * c.image_dim * 2)});
@@ -354,18 +372,22 @@ wan_status build_workspace(wan_dit* h) {
     return WAN_OK;
 }
 
-// RoPE cos/sin tables per axis, computed in double on the host.
+// RoPE cos/sin tables per axis, computed in double on the host; entry (pos, k)
+// at pos * pairs + k, or at k * len + pos when pair_major.
 void rope_tables_host(const wan_dit_config& c, int Fp, int Hp, int Wp, std::vector<float2>& out, int& nt, int& nh,
-                      int& nw) {
+                      int& nw, bool pair_major = false) {
     nt = c.rope_t / 2;
     nh = c.rope_h / 2;
     nw = c.rope_w / 2;
     out.clear();
     auto axis = [&](int len, int d_a) {
+        const size_t base = out.size();
+        out.resize(base + (size_t)len * (d_a / 2));
         for (int pos = 0; pos < len; ++pos)
             for (int k = 0; k < d_a / 2; ++k) {
                 const double ang = pos * std::pow((double)c.rope_theta, -2.0 * k / d_a);
-                out.push_back(make_float2((float)std::cos(ang), (float)std::sin(ang)));
+                const size_t at = pair_major ? (size_t)k * len + pos : (size_t)pos * (d_a / 2) + k;
+                out[base + at] = make_float2((float)std::cos(ang), (float)std::sin(ang));
             }
     };
     axis(Fp, c.rope_t);
@@ -375,156 +397,240 @@ void rope_tables_host(const wan_dit_config& c, int Fp, int Hp, int Wp, std::vect
 
 struct Shape {
     int B, F, Hz, Wz, Lc, per_token, lat_dtype, Li;  // Li: image tokens per sample, 0 without the image branch
+    int cfg_euler;  // 1: B = 2 CFG pair whose proj_out epilogue writes the Euler-updated latent
+    // sequence-parallel shard: this rank holds tokens [tok0, tok0 + Ls) of the
+    // global sequence padded to world * Ls (tokens >= L are padding); world 0: whole sequence
+    int tok0, Ls, world;
     int L() const { return F * (Hz / 2) * (Wz / 2); }
+    int rows_per_sample() const { return world ? Ls : L(); }
 };
 
-// Issue every launch of one forward on ctx.stream (eager or under capture).
-cudaError_t issue_forward(wan_dit* h, const Shape& s, const Plan& plan, const LaunchCtx& ctx, bool dump, KTimer* tm) {
-    const auto& c = h->cfg;
-    const int B = s.B, L = s.L(), Lc = s.Lc, D = c.dim, Fd = c.ffn_dim, N = c.num_blocks;
-    const int R = B * L, Rc = B * Lc;
-    const long long D6 = 6LL * D;
-    cudaError_t e;
 #define TRY(x)                               \
     do {                                     \
-        e = (x);                             \
-        if (e != cudaSuccess) return e;      \
+        cudaError_t e_ = (x);                \
+        if (e_ != cudaSuccess) return e_;    \
     } while (0)
 #define TRYK(kc, x)                          \
     do {                                     \
         if (tm) tm->begin(ctx.stream);       \
-        e = (x);                             \
-        if (e != cudaSuccess) return e;      \
+        cudaError_t e_ = (x);                \
+        if (e_ != cudaSuccess) return e_;    \
         if (tm) tm->end(ctx.stream, kc);     \
     } while (0)
-    auto epi = [](int kind, const float* bias, void* out, long long ldo) {
-        EpiParams p{};
-        p.kind = kind;
-        p.bias = bias;
-        p.out = out;
-        p.ldo = ldo;
-        p.mod_div = 1;
-        return p;
-    };
-    // ---- patch embedding: gather + GEMM (K = in_ch * 4)
-    TRYK(WAN_KC_PATCHIFY, wan::launch_patchify(h->lat_stage, s.lat_dtype, B, c.in_ch, s.F, s.Hz, s.Wz, h->X, h->Kp, ctx));
+
+EpiParams make_epi(int kind, const float* bias, void* out, long long ldo) {
+    EpiParams p{};
+    p.kind = kind;
+    p.bias = bias;
+    p.out = out;
+    p.ldo = ldo;
+    p.mod_div = 1;
+    return p;
+}
+
+// RMSNorm row factors from the per-head sums of squares (row stride 3 heads):
+// self-attention q | k, cross-attention q.
+wan::RowNorm row_norm(const wan_dit* h, int which) {
+    const auto& c = h->cfg;
+    return wan::RowNorm{h->ssq + which * c.heads, 3LL * c.heads, c.heads, 1.0f / c.dim, c.eps};
+}
+
+// Patchify, patch GEMM, timestep embedding, text embedding and the cross K/V of
+// every block (the part of the forward before the blocks).
+cudaError_t issue_prologue(wan_dit* h, const Shape& s, const LaunchCtx& ctx, bool dump, KTimer* tm) {
+    const auto& c = h->cfg;
+    const int B = s.B, Lr = s.rows_per_sample(), Lc = s.Lc, D = c.dim, N = c.num_blocks;
+    const int R = B * Lr, Rc = B * Lc;
+    const long long D6 = 6LL * D;
+    TRYK(WAN_KC_PATCHIFY, wan::launch_patchify(h->lat_stage, s.lat_dtype, B, c.in_ch, s.F, s.Hz, s.Wz, h->X, h->Kp, ctx,
+                                               s.world ? s.tok0 : 0, Lr));
     TRYK(WAN_KC_GEMM, wan::launch_gemm(h->X, h->Kp, h->w_pe_k, h->Kp, R, D, h->Kp,
-                         epi(wan::EPI_BIAS, h->b_pe, h->x, D), ctx));
+                                       make_epi(wan::EPI_BIAS, h->b_pe, h->x, D), ctx));
     if (dump) TRY(cudaMemcpyAsync(h->dump, h->x, (size_t)R * D * 2, cudaMemcpyDeviceToDevice, ctx.stream));
     // ---- timestep embedding -> temb [B|R, D] f32, tproj [B|R, 6D] f32
-    int mod_div;
     if (!s.per_token) {
         TRYK(WAN_KC_EMBEDDING, wan::launch_gemv(h->w_t1, h->b_t1, h->t_stage, 1, h->th32, D, B, D, c.freq_dim, 2, 1, ctx));
         TRYK(WAN_KC_EMBEDDING, wan::launch_gemv(h->w_t2, h->b_t2, h->th32, D, h->temb, D, B, D, D, 0, 0, ctx));
         TRYK(WAN_KC_EMBEDDING, wan::launch_gemv(h->w_tp, h->b_tp, h->temb, D, h->tproj, D6, B, 6 * D, D, 1, 0, ctx));
         TRYK(WAN_KC_EMBEDDING, wan::launch_mod_combine(h->sst_all, h->tproj, h->modc, N, B, D, ctx));
-        mod_div = L;
     } else {
         TRYK(WAN_KC_EMBEDDING, wan::launch_sinusoid_bf16(h->t_stage, R, c.freq_dim, h->tsin, ctx));
         TRYK(WAN_KC_GEMM, wan::launch_gemm(h->tsin, c.freq_dim, h->w_t1, c.freq_dim, R, D, c.freq_dim,
-                             epi(wan::EPI_BIAS_SILU, h->b_t1, h->y, D), ctx));
-        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, h->w_t2, D, R, D, D, epi(wan::EPI_BIAS_F32, h->b_t2, h->temb, D), ctx));
+                                           make_epi(wan::EPI_BIAS_SILU, h->b_t1, h->y, D), ctx));
+        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, h->w_t2, D, R, D, D, make_epi(wan::EPI_BIAS_F32, h->b_t2, h->temb, D), ctx));
         TRYK(WAN_KC_EMBEDDING, wan::launch_silu_bf16(h->temb, h->tsilu, (long long)R * D, ctx));
-        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->tsilu, D, h->w_tp, D, R, 6 * D, D, epi(wan::EPI_BIAS_F32, h->b_tp, h->tproj, D6), ctx));
-        mod_div = 1;
+        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->tsilu, D, h->w_tp, D, R, 6 * D, D,
+                                           make_epi(wan::EPI_BIAS_F32, h->b_tp, h->tproj, D6), ctx));
     }
     // ---- text embedding and the cross-attention keys/values of every block
     TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ctx_stage, c.text_dim, h->w_x1, c.text_dim, Rc, D, c.text_dim,
-                         epi(wan::EPI_BIAS_GELU, h->b_x1, h->th, D), ctx));
-    TRYK(WAN_KC_GEMM, wan::launch_gemm(h->th, D, h->w_x2, D, Rc, D, D, epi(wan::EPI_BIAS, h->b_x2, h->ctx, D), ctx));
+                                       make_epi(wan::EPI_BIAS_GELU, h->b_x1, h->th, D), ctx));
+    TRYK(WAN_KC_GEMM, wan::launch_gemm(h->th, D, h->w_x2, D, Rc, D, D, make_epi(wan::EPI_BIAS, h->b_x2, h->ctx, D), ctx));
     const long long ldkv = 2LL * N * D;
-    TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ctx, D, h->w_kv, D, Rc, (int)ldkv, D, epi(wan::EPI_BIAS, h->b_kv, h->kv, ldkv), ctx));
+    TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ctx, D, h->w_kv, D, Rc, (int)ldkv, D, make_epi(wan::EPI_BIAS, h->b_kv, h->kv, ldkv), ctx));
     TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rmsnorm_rope(h->kv, ldkv, Rc, D, c.eps, h->k2_gain, D, N, 2LL * D, nullptr, 0, ctx));
     // ---- image tokens (I2V): embedder (Linear, GELU_tanh, Linear), then every block's image K/V and key norm
     const int Ri = B * s.Li;
     if (s.Li > 0) {
         TRYK(WAN_KC_GEMM, wan::launch_gemm(h->img_stage, c.image_dim, h->w_i1, c.image_dim, Ri, D, c.image_dim,
-                             epi(wan::EPI_BIAS_GELU, h->b_i1, h->ih, D), ctx));
-        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ih, D, h->w_i2, D, Ri, D, D, epi(wan::EPI_BIAS, h->b_i2, h->ictx, D), ctx));
-        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ictx, D, h->w_kvi, D, Ri, (int)ldkv, D, epi(wan::EPI_BIAS, h->b_kvi, h->kvi, ldkv),
-                             ctx));
+                                           make_epi(wan::EPI_BIAS_GELU, h->b_i1, h->ih, D), ctx));
+        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ih, D, h->w_i2, D, Ri, D, D, make_epi(wan::EPI_BIAS, h->b_i2, h->ictx, D), ctx));
+        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->ictx, D, h->w_kvi, D, Ri, (int)ldkv, D,
+                                           make_epi(wan::EPI_BIAS, h->b_kvi, h->kvi, ldkv), ctx));
         TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rmsnorm_rope(h->kvi, ldkv, Ri, D, c.eps, h->ki_gain, D, N, 2LL * D, nullptr, 0,
                                                            ctx));
     }
+    return cudaSuccess;
+}
 
+// Block i up to the self-attention: norm1 + modulation (shift row 0, scale row 1),
+// the q, k, v projection with q and k RMSNorm'd across heads in two parts (the
+// epilogue stores gain * RoPE(q), gain * RoPE(k) and each head's sum of
+// squares; the key row factors are applied here in place, the query factors
+// inside the attention -- or here too when the queries leave the GPU).
+cudaError_t issue_block_pre(wan_dit* h, const Shape& s, const Plan& plan, int i, const LaunchCtx& ctx, KTimer* tm,
+                            bool normalize_q) {
+    const auto& c = h->cfg;
+    const int B = s.B, Lr = s.rows_per_sample(), D = c.dim;
+    const int R = B * Lr;
+    const long long D6 = 6LL * D;
+    const BlockW& w = h->blocks[i];
+    const float* mc = h->modc + (long long)i * B * 6 * D;
+    const int mod_div = s.per_token ? 1 : Lr;
+    // per-sample: precombined rows of modc (1 + scale folded in); per-token: table + projection rows
+    if (!s.per_token)
+        TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 2, nullptr, nullptr, nullptr, mc,
+                                                     nullptr, mc + D, mod_div, D6, ctx));
+    else
+        TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, w.sst, h->tproj,
+                                                     w.sst + D, h->tproj + D, mod_div, D6, ctx));
+    EpiParams p = make_epi(wan::EPI_QK_NORM, w.bqkv, h->qkv, 3LL * D);
+    p.norm_cols = 2 * D;
+    p.gain = w.qk_gain;
+    p.ssq = h->ssq;
+    p.ssq_ld = 3LL * c.heads;
+    p.rope_L = Lr;
+    p.rope_tok0 = s.world ? s.tok0 : 0;
+    p.rope = plan.rt;
+    TRYK(WAN_KC_GEMM_QKV, wan::launch_gemm(h->y, D, w.wqkv, D, R, 3 * D, D, p, ctx));
+    char* qkv = reinterpret_cast<char*>(h->qkv);
+    TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rms_apply(qkv + 2LL * D, 3LL * D, R, D, row_norm(h, 1), ctx));
+    if (normalize_q) TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rms_apply(qkv, 3LL * D, R, D, row_norm(h, 0), ctx));
+    return cudaSuccess;
+}
+
+// Block i after the self-attention, whose output (all heads) is in h->o: O
+// projection + gated residual, affine norm2, cross-attention with its q
+// RMSNorm split like the self-attention's, residual, norm3 + modulation,
+// GELU-tanh FFN, gated residual.
+cudaError_t issue_block_post(wan_dit* h, const Shape& s, int i, const LaunchCtx& ctx, KTimer* tm) {
+    const auto& c = h->cfg;
+    const int B = s.B, Lr = s.rows_per_sample(), Lc = s.Lc, D = c.dim, Fd = c.ffn_dim, N = c.num_blocks;
+    const int R = B * Lr;
+    const long long D6 = 6LL * D, ldkv = 2LL * N * D;
+    const BlockW& w = h->blocks[i];
+    const float* mc = h->modc + (long long)i * B * 6 * D;
+    const int mod_div = s.per_token ? 1 : Lr;
+    {
+        EpiParams p = make_epi(wan::EPI_GATE_RESIDUAL, w.bo, h->x, D);
+        p.gate0 = s.per_token ? w.sst + 2 * D : nullptr;
+        p.gate1 = s.per_token ? h->tproj + 2 * D : mc + 2 * D;
+        p.mod_div = mod_div;
+        p.mod_ld = D6;
+        TRYK(WAN_KC_GEMM_O, wan::launch_gemm(h->o, D, w.wo, D, R, D, D, p, ctx));
+    }
+    // 2. cross-attention: affine norm2, q projection + RMSNorm, attention to the context
+    TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 1, w.n2_g, w.n2_b, nullptr, nullptr, nullptr,
+                                                 nullptr, 1, 0, ctx));
+    {
+        EpiParams p = make_epi(wan::EPI_QK_NORM, w.bq2, h->qc, D);
+        p.norm_cols = D;
+        p.gain = w.q2_gain;
+        p.ssq = h->ssq + 2 * c.heads;
+        p.ssq_ld = 3LL * c.heads;
+        TRYK(WAN_KC_GEMM_Q2, wan::launch_gemm(h->y, D, w.wq2, D, R, D, D, p, ctx));
+    }
+    const wan::RowNorm rn_qc = row_norm(h, 2);
+    const char* kvb = reinterpret_cast<const char*>(h->kv) + 2LL * (2LL * i * D);
+    TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_attention(h->qc, D, kvb, ldkv, kvb + 2LL * D, ldkv, h->o, D, B, c.heads, Lr, Lc,
+                                                       ctx, rn_qc));
+    if (s.Li > 0) {  // image attention with the same queries, added before attn2.to_out
+        const char* kvib = reinterpret_cast<const char*>(h->kvi) + 2LL * (2LL * i * D);
+        TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_attention(h->qc, D, kvib, ldkv, kvib + 2LL * D, ldkv, h->o2, D, B,
+                                                           c.heads, Lr, s.Li, ctx, rn_qc));
+        TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_add_bf16(h->o, h->o2, (long long)R * D, ctx));
+    }
+    TRYK(WAN_KC_GEMM_O2, wan::launch_gemm(h->o, D, w.wo2, D, R, D, D, make_epi(wan::EPI_RESIDUAL, w.bo2, h->x, D), ctx));
+    // 3. feed-forward: norm3 + modulation (shift row 3, scale row 4), GELU-tanh, gated residual (row 5)
+    if (!s.per_token)
+        TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 2, nullptr, nullptr, nullptr, mc + 3 * D,
+                                                     nullptr, mc + 4 * D, mod_div, D6, ctx));
+    else
+        TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, w.sst + 3 * D,
+                                                     h->tproj + 3 * D, w.sst + 4 * D, h->tproj + 4 * D, mod_div, D6,
+                                                     ctx));
+    TRYK(WAN_KC_GEMM_FFN_UP, wan::launch_gemm(h->y, D, w.w1, D, R, Fd, D, make_epi(wan::EPI_BIAS_GELU, w.b1, h->u, Fd), ctx));
+    {
+        EpiParams p = make_epi(wan::EPI_GATE_RESIDUAL, w.b2, h->x, D);
+        p.gate0 = s.per_token ? w.sst + 5 * D : nullptr;
+        p.gate1 = s.per_token ? h->tproj + 5 * D : mc + 5 * D;
+        p.mod_div = mod_div;
+        p.mod_ld = D6;
+        TRYK(WAN_KC_GEMM_FFN_DOWN, wan::launch_gemm(h->u, Fd, w.w2, Fd, R, D, Fd, p, ctx));
+    }
+    return cudaSuccess;
+}
+
+// Output head: FP32 LayerNorm, (shift, scale) = head table + temb, proj_out with
+// the unpatchify scatter (or the fused CFG + Euler step) in its epilogue.
+cudaError_t issue_head(wan_dit* h, const Shape& s, const LaunchCtx& ctx, KTimer* tm) {
+    const auto& c = h->cfg;
+    const int B = s.B, L = s.L(), Lr = s.rows_per_sample(), D = c.dim;
+    const int R = B * Lr;
+    TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, h->sst_out, h->temb,
+                                                 h->sst_out + D, h->temb, s.per_token ? 1 : Lr, D, ctx));
+    EpiParams p = make_epi(s.cfg_euler ? wan::EPI_CFG_EULER : wan::EPI_UNPATCHIFY, h->b_po, h->vel_stage, 0);
+    p.L = L;
+    p.C = c.out_ch;
+    p.F = s.F;
+    p.Hz = s.Hz;
+    p.Wz = s.Wz;
+    p.up_rows = Lr;
+    p.up_tok0 = s.world ? s.tok0 : 0;
+    if (s.cfg_euler) {  // rows [0, L): conditional sample, [L, 2L): unconditional; x = sample 0's latent
+        p.pair_off = L;
+        p.x = h->lat_stage;
+        p.sched = h->sched;
+        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, h->w_po, D, L, c.out_ch * 4, D, p, ctx));
+    } else {
+        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, h->w_po, D, R, c.out_ch * 4, D, p, ctx));
+    }
+    return cudaSuccess;
+}
+
+// Issue every launch of one forward on ctx.stream (eager or under capture).
+cudaError_t issue_forward(wan_dit* h, const Shape& s, const Plan& plan, const LaunchCtx& ctx, bool dump, KTimer* tm) {
+    const auto& c = h->cfg;
+    const int B = s.B, L = s.L(), D = c.dim, N = c.num_blocks;
+    const int R = B * L;
+    TRY(issue_prologue(h, s, ctx, dump, tm));
     char* qkv = reinterpret_cast<char*>(h->qkv);
     for (int i = 0; i < N; ++i) {
-        const BlockW& w = h->blocks[i];
-        // 1. self-attention: norm1 + modulation (shift row 0, scale row 1)
-        // per-sample: precombined rows of modc (1 + scale folded in); per-token: table + projection rows
-        const float* mc = h->modc + (long long)i * B * 6 * D;
-        if (!s.per_token)
-            TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 2, nullptr, nullptr, nullptr, mc,
-                                                         nullptr, mc + D, mod_div, D6, ctx));
-        else
-            TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, w.sst, h->tproj,
-                                                         w.sst + D, h->tproj + D, mod_div, D6, ctx));
-        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, w.wqkv, D, R, 3 * D, D, epi(wan::EPI_BIAS, w.bqkv, h->qkv, 3LL * D), ctx));
-        TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rmsnorm_rope(h->qkv, 3LL * D, R, D, c.eps, w.qk_gain, D, 2, D, &plan.rt, L, ctx));
-        TRYK(WAN_KC_SELF_ATTENTION, wan::launch_attention(qkv, 3LL * D, qkv + 2LL * D, 3LL * D, qkv + 4LL * D, 3LL * D, h->o, D, B, c.heads, L,
-                                  L, ctx));
-        {
-            EpiParams p = epi(wan::EPI_GATE_RESIDUAL, w.bo, h->x, D);
-            p.gate0 = s.per_token ? w.sst + 2 * D : nullptr;
-            p.gate1 = s.per_token ? h->tproj + 2 * D : mc + 2 * D;
-            p.mod_div = mod_div;
-            p.mod_ld = D6;
-            TRYK(WAN_KC_GEMM, wan::launch_gemm(h->o, D, w.wo, D, R, D, D, p, ctx));
-        }
-        // 2. cross-attention: affine norm2, q projection + RMSNorm, attention to the context
-        TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 1, w.n2_g, w.n2_b, nullptr, nullptr, nullptr, nullptr, 1, 0,
-                                  ctx));
-        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, w.wq2, D, R, D, D, epi(wan::EPI_BIAS, w.bq2, h->qc, D), ctx));
-        TRYK(WAN_KC_RMSNORM_ROPE, wan::launch_rmsnorm_rope(h->qc, D, R, D, c.eps, w.q2_gain, D, 1, 0, nullptr, 0, ctx));
-        const char* kvb = reinterpret_cast<const char*>(h->kv) + 2LL * (2LL * i * D);
-        TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_attention(h->qc, D, kvb, ldkv, kvb + 2LL * D, ldkv, h->o, D, B, c.heads, L, Lc, ctx));
-        if (s.Li > 0) {  // image attention with the same queries, added before attn2.to_out
-            const char* kvib = reinterpret_cast<const char*>(h->kvi) + 2LL * (2LL * i * D);
-            TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_attention(h->qc, D, kvib, ldkv, kvib + 2LL * D, ldkv, h->o2, D, B,
-                                                               c.heads, L, s.Li, ctx));
-            TRYK(WAN_KC_CROSS_ATTENTION, wan::launch_add_bf16(h->o, h->o2, (long long)R * D, ctx));
-        }
-        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->o, D, w.wo2, D, R, D, D, epi(wan::EPI_RESIDUAL, w.bo2, h->x, D), ctx));
-        // 3. feed-forward: norm3 + modulation (shift row 3, scale row 4), GELU-tanh, gated residual (row 5)
-        if (!s.per_token)
-            TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 2, nullptr, nullptr, nullptr, mc + 3 * D,
-                                                         nullptr, mc + 4 * D, mod_div, D6, ctx));
-        else
-            TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, w.sst + 3 * D,
-                                                         h->tproj + 3 * D, w.sst + 4 * D, h->tproj + 4 * D, mod_div, D6,
-                                                         ctx));
-        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, w.w1, D, R, Fd, D, epi(wan::EPI_BIAS_GELU, w.b1, h->u, Fd), ctx));
-        {
-            EpiParams p = epi(wan::EPI_GATE_RESIDUAL, w.b2, h->x, D);
-            p.gate0 = s.per_token ? w.sst + 5 * D : nullptr;
-            p.gate1 = s.per_token ? h->tproj + 5 * D : mc + 5 * D;
-            p.mod_div = mod_div;
-            p.mod_ld = D6;
-            TRYK(WAN_KC_GEMM, wan::launch_gemm(h->u, Fd, w.w2, Fd, R, D, Fd, p, ctx));
-        }
+        TRY(issue_block_pre(h, s, plan, i, ctx, tm, false));
+        TRYK(WAN_KC_SELF_ATTENTION, wan::launch_attention(qkv, 3LL * D, qkv + 2LL * D, 3LL * D, qkv + 4LL * D, 3LL * D, h->o,
+                                                          D, B, c.heads, L, L, ctx, row_norm(h, 0)));
+        TRY(issue_block_post(h, s, i, ctx, tm));
         if (dump)
             TRY(cudaMemcpyAsync(reinterpret_cast<char*>(h->dump) + (size_t)(i + 1) * R * D * 2, h->x, (size_t)R * D * 2,
                                 cudaMemcpyDeviceToDevice, ctx.stream));
     }
-    // ---- head: FP32 LayerNorm, (shift, scale) = head table + temb, proj_out, unpatchify
-    TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, h->sst_out, h->temb, h->sst_out + D,
-                              h->temb, s.per_token ? 1 : L, D, ctx));
-    {
-        EpiParams p = epi(wan::EPI_UNPATCHIFY, h->b_po, h->vel_stage, 0);
-        p.L = L;
-        p.C = c.out_ch;
-        p.F = s.F;
-        p.Hz = s.Hz;
-        p.Wz = s.Wz;
-        TRYK(WAN_KC_GEMM, wan::launch_gemm(h->y, D, h->w_po, D, R, c.out_ch * 4, D, p, ctx));
-    }
+    return issue_head(h, s, ctx, tm);
+}
 #undef TRY
 #undef TRYK
-    return cudaSuccess;
-}
 
 wan_status ensure_plan(wan_dit* h, const Shape& s, Plan** out) {
-    PlanKey key{s.B, s.F, s.Hz, s.Wz, s.Lc, s.per_token, s.lat_dtype, s.Li};
+    PlanKey key{s.B, s.F, s.Hz, s.Wz, s.Lc, s.per_token, s.lat_dtype, s.Li, s.cfg_euler, s.world, s.tok0, s.Ls};
     auto it = h->plans.find(key);
     if (it != h->plans.end()) {
         *out = &it->second;
@@ -534,7 +640,9 @@ wan_status ensure_plan(wan_dit* h, const Shape& s, Plan** out) {
     std::vector<float2> tab;
     int nt, nh, nw;
     const int Fp = s.F, Hp = s.Hz / 2, Wp = s.Wz / 2;
-    rope_tables_host(h->cfg, Fp, Hp, Wp, tab, nt, nh, nw);
+    // the q/k projection epilogue reads the tables: pair-major, so the 32 tokens of
+    // a warp read neighbouring entries
+    rope_tables_host(h->cfg, Fp, Hp, Wp, tab, nt, nh, nw, true);
     WAN_CU(cudaMalloc(&plan.rope, tab.size() * sizeof(float2)), "rope table allocation");
     WAN_CU(cudaMemcpy(plan.rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice), "rope upload");
     plan.rt.t = plan.rope;
@@ -546,10 +654,13 @@ wan_status ensure_plan(wan_dit* h, const Shape& s, Plan** out) {
     plan.rt.nt = nt;
     plan.rt.nh = nh;
     plan.rt.nw = nw;
+    plan.rt.pair_major = 1;
     auto res = h->plans.emplace(key, plan);
     *out = &res.first->second;
     return WAN_OK;
 }
+
+wan_status run_plan(wan_dit* h, const Shape& s, Plan* plan, cudaStream_t st);
 
 LaunchCtx make_ctx(wan_dit* h, cudaStream_t st, int* counter) {
     LaunchCtx ctx;
@@ -803,7 +914,7 @@ wan_status wan_dit_forward_image(wan_dit* h, const void* latent, int latent_dtyp
     }
     cudaSetDevice(h->device);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    Shape s{B, F, Hz, Wz, Lc, per_token, latent_dtype, Li};
+    Shape s{B, F, Hz, Wz, Lc, per_token, latent_dtype, Li, 0, 0, 0, 0};
     Plan* plan = nullptr;
     wan_status ps = ensure_plan(h, s, &plan);
     if (ps != WAN_OK) return ps;
@@ -816,6 +927,21 @@ wan_status wan_dit_forward_image(wan_dit* h, const void* latent, int latent_dtyp
     WAN_CU(cudaMemcpyAsync(h->ctx_stage, context, (size_t)B * Lc * c.text_dim * 2, h2d, st), "context copy");
     if (Li > 0) WAN_CU(cudaMemcpyAsync(h->img_stage, image, (size_t)B * Li * c.image_dim * 2, h2d, st), "image copy");
 
+    WAN_CU_RET(run_plan(h, s, plan, st));
+    const size_t vel_bytes = (size_t)B * c.out_ch * F * Hz * Wz * 4;
+    WAN_CU(cudaMemcpyAsync(velocity, h->vel_stage, vel_bytes, io_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+                           st),
+           "velocity copy");
+    return WAN_OK;
+}
+
+}  // extern "C"
+
+namespace {
+// Launch the forward of plan `plan` on `st` (graph replay, or eager launches
+// when graphs are off or the block dump is on).  Inputs are already staged.
+wan_status run_plan(wan_dit* h, const Shape& s, Plan* plan, cudaStream_t st) {
+    const auto& c = h->cfg;
     const bool dump = h->dump != nullptr;
     const bool timed = h->timing;
     if (timed) WAN_CU(plan->timer.ensure(20 * c.num_blocks + 64), "timing events");
@@ -853,10 +979,190 @@ wan_status wan_dit_forward_image(wan_dit* h, const void* latent, int latent_dtyp
     }
     h->last_plan = plan;
     h->last_timed = timed;
-    const size_t vel_bytes = (size_t)B * c.out_ch * F * Hz * Wz * 4;
+    return WAN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+wan_status wan_dit_forward_cfg_euler(wan_dit* h, const float* x, int F, int Hz, int Wz, float timestep,
+                                     const void* context, int Lc, float guidance, float sigma, float sigma_next,
+                                     float* x_next, int io_on_device, void* stream) {
+    if (!h) return WAN_EINVAL;
+    if (!x || !context || !x_next) return fail(h, WAN_EINVAL, "null input or output pointer");
+    const auto& c = h->cfg;
+    if (c.in_ch != c.out_ch) return fail(h, WAN_EUNSUPPORTED, "the sampler step needs in_ch == out_ch");
+    if (c.max_batch < 2) return fail(h, WAN_ESHAPE, "the CFG pair needs max_batch >= 2");
+    if (F < 1 || Hz < 2 || Wz < 2 || Hz % 2 || Wz % 2) return fail(h, WAN_ESHAPE, "latent grid must be F>=1, even Hz, Wz");
+    const long long L = (long long)F * (Hz / 2) * (Wz / 2);
+    if (L > c.max_tokens) return fail(h, WAN_ESHAPE, "token count exceeds max_tokens");
+    if (Lc < 1 || Lc > c.max_text) return fail(h, WAN_ESHAPE, "context length outside 1..max_text");
+    if (!std::isfinite(guidance) || !std::isfinite(sigma) || !std::isfinite(sigma_next) || !std::isfinite(timestep))
+        return fail(h, WAN_EINVAL, "non-finite sampler scalar");
+    if (h->loaded.empty()) return fail(h, WAN_ENOWEIGHTS, "forward before load_weights");
+    if (h->loaded.size() != h->slots.size()) {
+        char buf[256];
+        int m = wan_dit_missing_weights(h, buf, sizeof(buf));
+        return fail(h, WAN_EMISSING_WEIGHT, std::to_string(m) + " weights missing: " + buf);
+    }
+    cudaSetDevice(h->device);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Shape s{2, F, Hz, Wz, Lc, 0, WAN_DTYPE_F32, 0, 1, 0, 0, 0};
+    Plan* plan = nullptr;
+    wan_status ps = ensure_plan(h, s, &plan);
+    if (ps != WAN_OK) return ps;
+    // the same latent for both samples; per-call scalars through a tiny kernel
+    const cudaMemcpyKind h2d = io_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    const size_t lat_bytes = (size_t)c.in_ch * F * Hz * Wz * 4;
+    WAN_CU(cudaMemcpyAsync(h->lat_stage, x, lat_bytes, h2d, st), "latent copy");
+    WAN_CU(cudaMemcpyAsync(reinterpret_cast<char*>(h->lat_stage) + lat_bytes, x, lat_bytes, h2d, st), "latent copy");
+    WAN_CU(cudaMemcpyAsync(h->ctx_stage, context, (size_t)2 * Lc * c.text_dim * 2, h2d, st), "context copy");
+    LaunchCtx sctx = make_ctx(h, st, nullptr);
+    WAN_CU(wan::launch_set_sampler_scalars(h->sched, guidance, sigma_next - sigma, h->t_stage, 2, timestep, sctx),
+           "sampler scalars");
+    WAN_CU_RET(run_plan(h, s, plan, st));
+    WAN_CU(cudaMemcpyAsync(x_next, h->vel_stage, lat_bytes, io_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+                           st),
+           "latent copy back");
+    return WAN_OK;
+}
+
+// ---------------------------------------------------------------- sequence-parallel (Ulysses) stages
+static Shape sp_shape(const wan_dit* h) {
+    return Shape{h->sp_B, h->sp_F, h->sp_Hz, h->sp_Wz, h->sp_Lc, h->sp_per_token, h->sp_dtype, 0, 0,
+                 h->sp_rank * h->sp_Ls, h->sp_Ls, h->sp_world};
+}
+
+wan_status wan_dit_sp_begin(wan_dit* h, const void* latent, int latent_dtype, int B, int F, int Hz, int Wz,
+                            const float* timestep, int per_token, const void* context, int Lc, int rank, int world,
+                            int io_on_device, void* stream) {
+    if (!h) return WAN_EINVAL;
+    if (!latent || !timestep || !context) return fail(h, WAN_EINVAL, "null input pointer");
+    if (latent_dtype != WAN_DTYPE_F32 && latent_dtype != WAN_DTYPE_BF16) return fail(h, WAN_EINVAL, "latent dtype");
+    const auto& c = h->cfg;
+    if (world < 1 || rank < 0 || rank >= world) return fail(h, WAN_EINVAL, "rank outside 0..world-1");
+    if (c.heads % world) return fail(h, WAN_ESHAPE, "heads must be a multiple of the world size");
+    if (c.image_dim > 0) return fail(h, WAN_EUNSUPPORTED, "the sequence-parallel stages cover text-to-video models");
+    if (B < 1 || B > c.max_batch) return fail(h, WAN_ESHAPE, "batch outside 1..max_batch");
+    if (F < 1 || Hz < 2 || Wz < 2 || Hz % 2 || Wz % 2) return fail(h, WAN_ESHAPE, "latent grid must be F>=1, even Hz, Wz");
+    if (Lc < 1 || Lc > c.max_text) return fail(h, WAN_ESHAPE, "context length outside 1..max_text");
+    if (per_token != 0 && per_token != 1) return fail(h, WAN_EINVAL, "per_token must be 0 or 1");
+    const long long L = (long long)F * (Hz / 2) * (Wz / 2);
+    const long long Ls = (L + world - 1) / world;  // the sequence padded to world * Ls tokens
+    if (Ls > c.max_tokens) return fail(h, WAN_ESHAPE, "shard tokens exceed max_tokens");
+    if (h->loaded.empty()) return fail(h, WAN_ENOWEIGHTS, "forward before load_weights");
+    if (h->loaded.size() != h->slots.size()) return fail(h, WAN_EMISSING_WEIGHT, "weights missing");
+    cudaSetDevice(h->device);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    h->sp_B = B; h->sp_F = F; h->sp_Hz = Hz; h->sp_Wz = Wz; h->sp_Lc = Lc; h->sp_per_token = per_token;
+    h->sp_dtype = latent_dtype; h->sp_rank = rank; h->sp_world = world; h->sp_Ls = (int)Ls;
+    const Shape s = sp_shape(h);
+    Plan* plan = nullptr;
+    wan_status ps = ensure_plan(h, s, &plan);
+    if (ps != WAN_OK) return ps;
+    const cudaMemcpyKind h2d = io_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    const size_t lat_bytes = (size_t)B * c.in_ch * F * Hz * Wz * (latent_dtype == WAN_DTYPE_F32 ? 4 : 2);
+    WAN_CU(cudaMemcpyAsync(h->lat_stage, latent, lat_bytes, h2d, st), "latent copy");
+    if (per_token) {  // this shard's columns of the [B, L] timesteps; padding tokens get t = 0
+        const long long tok0 = (long long)rank * Ls, n = std::max(0LL, std::min(Ls, L - tok0));
+        WAN_CU(cudaMemsetAsync(h->t_stage, 0, (size_t)B * Ls * 4, st), "timestep clear");
+        if (n > 0)
+            WAN_CU(cudaMemcpy2DAsync(h->t_stage, (size_t)Ls * 4, timestep + tok0, (size_t)L * 4, (size_t)n * 4, B, h2d, st),
+                   "timestep copy");
+    } else {
+        WAN_CU(cudaMemcpyAsync(h->t_stage, timestep, (size_t)B * 4, h2d, st), "timestep copy");
+    }
+    WAN_CU(cudaMemcpyAsync(h->ctx_stage, context, (size_t)B * Lc * c.text_dim * 2, h2d, st), "context copy");
+    LaunchCtx ctx = make_ctx(h, st, nullptr);
+    cudaError_t e = issue_prologue(h, s, ctx, false, nullptr);
+    if (e != cudaSuccess) return cuda_fail(h, e, "sequence-parallel prologue");
+    h->sp_active = true;
+    h->sp_next_block = 0;
+    h->sp_phase = 0;
+    return WAN_OK;
+}
+
+wan_status wan_dit_sp_block_qkv(wan_dit* h, int block, void* send, void* stream) {
+    if (!h) return WAN_EINVAL;
+    if (!send) return fail(h, WAN_EINVAL, "null send buffer");
+    if (!h->sp_active || block != h->sp_next_block || h->sp_phase != 0)
+        return fail(h, WAN_EINVAL, "sp_block_qkv out of order (sp_begin, then per block qkv and finish)");
+    cudaSetDevice(h->device);
+    const Shape s = sp_shape(h);
+    Plan* plan = nullptr;
+    wan_status ps = ensure_plan(h, s, &plan);
+    if (ps != WAN_OK) return ps;
+    LaunchCtx ctx = make_ctx(h, reinterpret_cast<cudaStream_t>(stream), nullptr);
+    cudaError_t e = issue_block_pre(h, s, *plan, block, ctx, nullptr, true);
+    if (e == cudaSuccess) e = wan::launch_sp_pack(h->qkv, send, s.B, s.world, s.Ls, h->cfg.dim, ctx);
+    if (e != cudaSuccess) return cuda_fail(h, e, "sequence-parallel block (q, k, v)");
+    h->sp_phase = 1;
+    return WAN_OK;
+}
+
+wan_status wan_dit_sp_attention(wan_dit* h, const void* recv, void* out, void* stream) {
+    if (!h) return WAN_EINVAL;
+    if (!recv || !out) return fail(h, WAN_EINVAL, "null exchange buffer");
+    if (!h->sp_active || h->sp_phase != 1) return fail(h, WAN_EINVAL, "sp_attention outside a block");
+    cudaSetDevice(h->device);
+    const Shape s = sp_shape(h);
+    const int hl = h->cfg.heads / s.world, hd = 128 * hl, Lp = s.Ls * s.world;
+    LaunchCtx ctx = make_ctx(h, reinterpret_cast<cudaStream_t>(stream), nullptr);
+    // queries: every (padded) token; keys: the L real tokens (padding sits past them).
+    // One launch per sample: a sample's keys are L rows of a buffer whose samples are Lp rows apart.
+    for (int b = 0; b < s.B; ++b) {
+        const char* r = reinterpret_cast<const char*>(recv) + (size_t)b * Lp * 3 * hd * 2;
+        char* o = reinterpret_cast<char*>(out) + (size_t)b * Lp * hd * 2;
+        cudaError_t e = wan::launch_attention(r, 3LL * hd, r + 2LL * hd, 3LL * hd, r + 4LL * hd, 3LL * hd, o, hd, 1, hl,
+                                              Lp, s.L(), ctx);
+        if (e != cudaSuccess) return cuda_fail(h, e, "sequence-parallel attention");
+    }
+    return WAN_OK;
+}
+
+wan_status wan_dit_sp_block_finish(wan_dit* h, int block, const void* back, void* stream) {
+    if (!h) return WAN_EINVAL;
+    if (!back) return fail(h, WAN_EINVAL, "null exchange buffer");
+    if (!h->sp_active || block != h->sp_next_block || h->sp_phase != 1)
+        return fail(h, WAN_EINVAL, "sp_block_finish out of order");
+    cudaSetDevice(h->device);
+    const Shape s = sp_shape(h);
+    LaunchCtx ctx = make_ctx(h, reinterpret_cast<cudaStream_t>(stream), nullptr);
+    cudaError_t e = wan::launch_sp_unpack(back, h->o, s.B, s.world, s.Ls, h->cfg.dim, ctx);
+    if (e == cudaSuccess) e = issue_block_post(h, s, block, ctx, nullptr);
+    if (e != cudaSuccess) return cuda_fail(h, e, "sequence-parallel block (output side)");
+    h->sp_phase = 0;
+    h->sp_next_block = block + 1;
+    return WAN_OK;
+}
+
+wan_status wan_dit_sp_end(wan_dit* h, float* velocity, int io_on_device, void* stream) {
+    if (!h) return WAN_EINVAL;
+    if (!velocity) return fail(h, WAN_EINVAL, "null output pointer");
+    if (!h->sp_active || h->sp_phase != 0 || h->sp_next_block != h->cfg.num_blocks)
+        return fail(h, WAN_EINVAL, "sp_end before every block finished");
+    cudaSetDevice(h->device);
+    const Shape s = sp_shape(h);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t vel_bytes = (size_t)s.B * h->cfg.out_ch * s.F * s.Hz * s.Wz * 4;
+    WAN_CU(cudaMemsetAsync(h->vel_stage, 0, vel_bytes, st), "velocity clear");
+    LaunchCtx ctx = make_ctx(h, st, nullptr);
+    cudaError_t e = issue_head(h, s, ctx, nullptr);
+    if (e != cudaSuccess) return cuda_fail(h, e, "sequence-parallel head");
     WAN_CU(cudaMemcpyAsync(velocity, h->vel_stage, vel_bytes, io_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
                            st),
            "velocity copy");
+    h->sp_active = false;
+    return WAN_OK;
+}
+
+wan_status wan_flow_sigmas(int steps, double shift, double* sigmas) {
+    if (!sigmas || steps < 1 || !(shift > 0.0) || !std::isfinite(shift)) return WAN_EINVAL;
+    for (int i = 0; i < steps; ++i) {
+        const double u = 1.0 - (double)i / steps;
+        sigmas[i] = shift * u / (1.0 + (shift - 1.0) * u);
+    }
+    sigmas[steps] = 0.0;
     return WAN_OK;
 }
 
@@ -952,7 +1258,7 @@ wan_status wan_op_sync(void* stream) {
 wan_status wan_op_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, int M, int N, int K, int epilogue,
                        const wan_epilogue* ep, void* stream) {
     if (!A || !W || !ep || !ep->out) return WAN_EINVAL;
-    if (epilogue < WAN_EPI_BIAS || epilogue > WAN_EPI_UNPATCHIFY) return WAN_EINVAL;
+    if ((epilogue < WAN_EPI_BIAS || epilogue > WAN_EPI_UNPATCHIFY) && epilogue != WAN_EPI_QK_NORM) return WAN_EINVAL;
     if (epilogue == WAN_EPI_GATE_RESIDUAL && !ep->gate0 && !ep->gate1) return WAN_EINVAL;
     if (M < 0) return WAN_ESHAPE;
     EpiParams p{};
@@ -973,9 +1279,73 @@ wan_status wan_op_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, i
         p.L = ep->up_F * (ep->up_Hz / 2) * (ep->up_Wz / 2);
         if (M % p.L) return WAN_ESHAPE;
     }
+    float2* tab = nullptr;
+    if (epilogue == WAN_EPI_QK_NORM) {
+        if (!ep->ssq || (ep->norm_cols > 0 && !ep->gain)) return WAN_EINVAL;
+        p.norm_cols = ep->norm_cols;
+        p.gain = ep->gain;
+        p.ssq = ep->ssq;
+        p.ssq_ld = ep->ssq_ld;
+        if (ep->rope) {
+            if (ep->rope_F <= 0 || ep->rope_H <= 0 || ep->rope_W <= 0 || ep->rope_t % 2 || ep->rope_h % 2 ||
+                ep->rope_w % 2 || ep->rope_t + ep->rope_h + ep->rope_w != 128 || !(ep->rope_theta > 0.f))
+                return WAN_ESHAPE;
+            if (N % 256 || ep->norm_cols % 128 || ep->norm_cols > N || ep->ssq_ld < ep->norm_cols / 128 ||
+                ep->ldo % 8)
+                return WAN_ESHAPE;
+            wan_dit_config c{};
+            c.rope_t = ep->rope_t;
+            c.rope_h = ep->rope_h;
+            c.rope_w = ep->rope_w;
+            c.rope_theta = ep->rope_theta;
+            std::vector<float2> host;
+            int nt, nh, nw;
+            rope_tables_host(c, ep->rope_F, ep->rope_H, ep->rope_W, host, nt, nh, nw, true);
+            if (cudaMalloc(&tab, host.size() * sizeof(float2)) != cudaSuccess) {
+                cudaGetLastError();
+                return WAN_ENOMEM;
+            }
+            if (cudaMemcpy(tab, host.data(), host.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess) {
+                cudaFree(tab);
+                return WAN_ECUDA;
+            }
+            p.rope = wan::RopeTables{tab, tab + (size_t)ep->rope_F * nt, tab + (size_t)ep->rope_F * nt + (size_t)ep->rope_H * nh,
+                                     ep->rope_F, ep->rope_H, ep->rope_W, nt, nh, nw, 1};
+            p.rope_L = ep->rope_F * ep->rope_H * ep->rope_W;
+        }
+    }
+    LaunchCtx ctx;
+    if (!op_ctx(reinterpret_cast<cudaStream_t>(stream), &ctx)) {
+        if (tab) cudaFree(tab);
+        return WAN_ECUDA;
+    }
+    cudaError_t e = wan::launch_gemm(A, lda, W, ldw, M, N, K, p, ctx);
+    if (tab) {  // the table is freed once the kernel that reads it has run
+        cudaStreamSynchronize(ctx.stream);
+        cudaFree(tab);
+    }
+    return op_status(e);
+}
+
+wan_status wan_op_attention_qnorm(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv,
+                                  void* o, int64_t ldo, int B, int heads, int Lq, int Lk, const float* q_ssq,
+                                  int64_t ssq_ld, int ngroups, float eps, void* stream) {
+    if (!q || !k || !v || !o || !q_ssq) return WAN_EINVAL;
+    if (B < 0 || heads <= 0 || Lq < 0 || Lk <= 0 || ngroups <= 0 || ssq_ld < ngroups) return WAN_ESHAPE;
     LaunchCtx ctx;
     if (!op_ctx(reinterpret_cast<cudaStream_t>(stream), &ctx)) return WAN_ECUDA;
-    return op_status(wan::launch_gemm(A, lda, W, ldw, M, N, K, p, ctx));
+    const wan::RowNorm rn{q_ssq, ssq_ld, ngroups, 1.0f / (128.0f * heads), eps};
+    return op_status(wan::launch_attention(q, ldq, k, ldk, v, ldv, o, ldo, B, heads, Lq, Lk, ctx, rn));
+}
+
+wan_status wan_op_rms_apply(void* buf, int64_t ld, int rows, int D, const float* ssq, int64_t ssq_ld, int ngroups,
+                            float eps, void* stream) {
+    if (!buf || !ssq) return WAN_EINVAL;
+    if (ngroups <= 0 || ssq_ld < ngroups || rows < 0 || D <= 0) return WAN_ESHAPE;
+    LaunchCtx ctx;
+    if (!op_ctx(reinterpret_cast<cudaStream_t>(stream), &ctx)) return WAN_ECUDA;
+    const wan::RowNorm rn{ssq, ssq_ld, ngroups, 1.0f / D, eps};
+    return op_status(wan::launch_rms_apply(buf, ld, rows, D, rn, ctx));
 }
 
 wan_status wan_op_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv, void* o,
@@ -1025,7 +1395,7 @@ wan_status wan_op_rmsnorm_rope(void* buf, int64_t ld, int rows, int D, float eps
         cudaFree(d);
         return WAN_ECUDA;
     }
-    wan::RopeTables rt{d, d + (size_t)Fp * nt, d + (size_t)Fp * nt + (size_t)Hp * nh, Fp, Hp, Wp, nt, nh, nw};
+    wan::RopeTables rt{d, d + (size_t)Fp * nt, d + (size_t)Fp * nt + (size_t)Hp * nh, Fp, Hp, Wp, nt, nh, nw, 0};
     cudaError_t e = wan::launch_rmsnorm_rope(buf, ld, rows, D, eps, gain, 0, 1, 0, &rt, Fp * Hp * Wp, ctx);
     cudaStreamSynchronize(ctx.stream);
     cudaFree(d);
@@ -1082,6 +1452,25 @@ wan_status wan_op_causal_conv3d(const void* x, const void* cache, int nc, int B,
     p.ldo = Co;
     p.mod_div = 1;
     return op_status(wan::launch_gemm(col, Kp, w, Kp, (int)M, Co, (int)Kp, p, ctx));
+}
+
+wan_status wan_op_conv3d(const void* x, const void* cache, int nc, int B, int T, int H, int W, int Ci, const void* w,
+                         int64_t ldw, const float* bias, int Co, int Co_pad, int kt, int kh, int kw, void* y, int64_t ldy,
+                         const void* add, int64_t ldadd, int time_split, void* stream) {
+    if (!x || !w || !y) return WAN_EINVAL;
+    if (B <= 0 || T <= 0 || H <= 0 || W <= 0 || Ci <= 0 || Co <= 0) return WAN_ESHAPE;
+    if (time_split && add) return WAN_EINVAL;
+    wan::ConvEpi e{};
+    e.kind = time_split ? wan::CONV_EPI_TIME_SPLIT : (add ? wan::CONV_EPI_ADD : wan::CONV_EPI_BIAS);
+    e.bias = bias;
+    e.y = reinterpret_cast<__nv_bfloat16*>(y);
+    e.ldy = ldy;
+    e.add = reinterpret_cast<const __nv_bfloat16*>(add);
+    e.ldadd = ldadd;
+    e.csplit = time_split ? Co / 2 : 0;
+    LaunchCtx ctx;
+    if (!op_ctx(reinterpret_cast<cudaStream_t>(stream), &ctx)) return WAN_ECUDA;
+    return op_status(wan::launch_conv3d(x, cache, nc, B, T, H, W, Ci, w, ldw, Co, Co_pad, kt, kh, kw, e, ctx));
 }
 
 wan_status wan_op_unpatchify(const float* rows, int B, int C, int F, int Hz, int Wz, float* velocity, void* stream) {

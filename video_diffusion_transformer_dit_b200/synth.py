@@ -138,3 +138,73 @@ def make_timestep_per_token(B, L, tokens_first_frame, seed=0) -> torch.Tensor:
     t = torch.rand(B, L, generator=g, dtype=torch.float32) * 1000.0
     t[:, :tokens_first_frame] = 0.0
     return t
+
+
+# ---------------------------------------------------------------- Wan2.1 VAE decoder
+VAE_DIMS = (384, 384, 384, 192, 96)    # conv_in width, then the up blocks' widths
+
+
+def vae_param_shapes(z_dim: int = 16) -> Dict[str, Tuple[int, ...]]:
+    """Names and shapes of the decoder parameters (post_quant_conv, conv_in, mid
+    block, four up blocks of three residual blocks, upsamplers, head)."""
+    s: Dict[str, Tuple[int, ...]] = {}
+
+    def conv(n, cin, cout, k):
+        s[n + ".weight"] = (cout, cin) + tuple(k)
+        s[n + ".bias"] = (cout,)
+
+    def norm(n, c):
+        s[n + ".gamma"] = (c,)
+        s[n + ".bias"] = (c,)
+
+    def res(n, cin, cout):
+        norm(n + ".norm1", cin)
+        conv(n + ".conv1", cin, cout, (3, 3, 3))
+        norm(n + ".norm2", cout)
+        conv(n + ".conv2", cout, cout, (3, 3, 3))
+        if cin != cout:
+            conv(n + ".conv_shortcut", cin, cout, (1, 1, 1))
+
+    d = VAE_DIMS
+    conv("post_quant_conv", z_dim, z_dim, (1, 1, 1))
+    conv("decoder.conv_in", z_dim, d[0], (3, 3, 3))
+    res("decoder.mid_block.resnets.0", d[0], d[0])
+    a = "decoder.mid_block.attentions.0"
+    norm(a + ".norm", d[0])
+    s[a + ".to_qkv.weight"] = (3 * d[0], d[0], 1, 1)
+    s[a + ".to_qkv.bias"] = (3 * d[0],)
+    s[a + ".proj.weight"] = (d[0], d[0], 1, 1)
+    s[a + ".proj.bias"] = (d[0],)
+    res("decoder.mid_block.resnets.1", d[0], d[0])
+    for i in range(4):
+        cin, cout = d[i] if i == 0 else d[i] // 2, d[i + 1]
+        for r in range(3):
+            res(f"decoder.up_blocks.{i}.resnets.{r}", cin if r == 0 else cout, cout)
+        if i < 3:
+            u = f"decoder.up_blocks.{i}.upsamplers.0"
+            s[u + ".resample.1.weight"] = (cout // 2, cout, 3, 3)
+            s[u + ".resample.1.bias"] = (cout // 2,)
+            if i < 2:
+                conv(u + ".time_conv", cout, 2 * cout, (3, 1, 1))
+    norm("decoder.norm_out", d[4])
+    conv("decoder.conv_out", d[4], 3, (3, 3, 3))
+    return s
+
+
+def make_vae_weights(seed=0, device="cpu") -> Dict[str, torch.Tensor]:
+    """Random decoder parameters, float32: weights N(0, 1) / sqrt(fan_in) rounded
+    to bf16 values, biases N(0, 0.1^2), norm gains 1 + N(0, 0.1^2)."""
+    out = {}
+    for name, shape in vae_param_shapes().items():
+        z = _randn(shape, seed, name, device)
+        if name.endswith(".weight"):
+            fan = 1
+            for v in shape[1:]:
+                fan *= v
+            out[name] = (z / math.sqrt(max(1, fan))).to(torch.bfloat16).to(torch.float32)
+        elif name.endswith(".gamma"):
+            out[name] = 1.0 + 0.1 * z
+        else:
+            out[name] = 0.1 * z
+    return out
+
