@@ -201,6 +201,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = configs.workload(args.workload)
     cfg = w["cfg"]
+    if args.blocks:
+        cfg["num_blocks"] = args.blocks
     B, Cc, F, Hz, Wz = w["latent"]
     L = F * (Hz // 2) * (Wz // 2)
     Lc = w["text_len"]
@@ -304,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic latents/contexts, random-init bf16 weights of the named shapes",
-        "config": arm_config(args.workload, world),
+        "config": dict(arm_config(args.workload, world), **({"blocks": args.blocks} if args.blocks else {})),
         "tflops_per_step": flops / 1e12,
         "achieved_tflops": flops / (ms * 1e-3) / 1e12,
         "tc_peak_frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
@@ -473,6 +475,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--blocks", type=int, default=None,
+                    help="profiling aid: run the workload's shapes with this many blocks (the line then says so "
+                         "in config.blocks; not a measurement of the named model)")
     ap.add_argument("--kernel", choices=KERNELS, default=None,
                     help="time one kernel alone at the workload's shapes (profiling aid)")
     args = ap.parse_args()

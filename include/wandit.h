@@ -220,7 +220,9 @@ WANDIT_API wan_status wan_flow_sigmas(int steps, double shift, double* sigmas);
  *   back   [B][world][Ls][hd]     slot j: head group j's output for this shard
  * sp_begin takes the whole latent, the whole timestep ([B] or [B, L]) and the
  * context, host or device like wan_dit_forward; it needs heads % world == 0,
- * Ls <= max_tokens and a text-to-video model.  sp_end writes the full-size
+ * Ls <= max_tokens (the workspace holds the shard) and a text-to-video model;
+ * the first sp_begin of a latent size allocates device staging for the whole
+ * latent and velocity (kept by the handle).  sp_end writes the full-size
  * velocity [B, out_ch, F, Hz, Wz] holding this shard's tokens and zeros
  * elsewhere: the sum over ranks is the velocity.  Calls are eager (no graph)
  * and asynchronous on `stream`; out-of-order calls return WAN_EINVAL.       */

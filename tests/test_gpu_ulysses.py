@@ -69,6 +69,7 @@ def test_sequence_parallel_stage_order_is_checked():
     cfg, W, lat, t, ctx, L = _case(False, seed=30)
     Ls, _ = U.shard(L, 2)
     r = U.SpRank(make_dit(cfg, 2, Ls, ctx.shape[1], {k: v.cuda() for k, v in W.items()}), 0, 2)
+    r.send = torch.empty(2, 2, Ls, 3 * r.hd, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(WanError) as e:          # a block before sp_begin
         r.block_qkv(0)
     assert e.value.name == "WAN_EINVAL"

@@ -5,29 +5,27 @@
 //
 // One CTA per (256 queries = two 128-row tiles, head, batch), 12 warps in
 // three warpgroups; the first gives registers to the two softmax groups
-// (96 / 200 / 200 per thread, 63488 of the 64512 = 384 threads x 168 at launch):
+// (88 / 208 / 208 per thread, 64512 in all = 384 threads x 168 at launch):
 //   warp 0      TMA producer: both Q tiles once, then K and V tiles of 128
 //               keys in two-slot rings (3-D tensor maps: rows past the
 //               sequence read as zero);
-//   warp 1      tensor-memory owner and MMA issuer;
+//   warp 1      tensor-memory owner and MMA issuer.  Tensor memory holds
+//               S0 | S1 | O0 | O1 (4 x 128 fp32 columns).  Per key tile j it
+//               issues  PV0(j-1) S0(j) PV1(j-1) S1(j)  in that order, so the
+//               commit that publishes S_t(j) also covers PV_t(j-1); each P.V
+//               goes in two K = 64 halves, the first as soon as the softmax
+//               has stored the probabilities of keys 0..63;
 //   warps 2..3  idle;
-//   warps 4..7  softmax of query tile 0, warps 8..11 of tile 1 (one query row
-//               per thread).
-// The keys are walked in sub-steps of 64 (two per K/V tile).  Tensor memory
-// holds S0a | S0b | S1a | S1b (64 fp32 columns each: every query tile has two
-// S buffers used by alternate sub-steps) | O0 | O1 (128 columns each).  While
-// the softmax of tile t works on S_t(s), the tensor core already computes
-// S_t(s + 1) into the other buffer, so the softmax warps run back to back
-// instead of waiting for the next S after each P.V.  Per sub-step s the issuer
-// runs  PV_0(s) S_0(s + 2) PV_1(s) S_1(s + 2):  S_t(s + 2) reuses the buffer of
-// S_t(s), whose probabilities P_t(s) (bf16, written by the softmax over its
-// own S columns) PV_t(s) has just read -- tcgen05 MMAs of one thread run in
-// issue order.  The softmax: tcgen05.ld of the 64-column S row, running max /
-// sum in fp32 (log2 domain), probabilities packed to bf16 and stored with
-// tcgen05.st; O is rescaled in TMEM only when a row maximum grows by more than
-// 2^8 (the stale maximum is exact because the final division uses the same
-// running sum), after the previous P.V of the tile has landed; at the end each
-// row is divided by its sum and stored as bf16.
+//   warps 4..7  softmax of tile 0, warps 8..11 softmax of tile 1 (one query
+//               row per thread, the two groups ping-pong with the tensor
+//               core): tcgen05.ld of the S row, running max / sum in fp32
+//               (log2 domain), probabilities packed to bf16 and written back
+//               with tcgen05.st over the S columns they came from (P aliases
+//               S), read there by the P.V MMA as its A operand.  O is
+//               rescaled in TMEM only when a row maximum grows by more than
+//               2^8 (the stale maximum is exact because the final division
+//               uses the same running sum); at the end each row is divided by
+//               its sum and stored as bf16.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -45,9 +43,7 @@ struct AttnParams {
 namespace attn {
 constexpr int TILE_BYTES = 128 * 128 * 2;  // one 128 x 128 bf16 tile = two 64-column swizzled halves
 constexpr int HALF_BYTES = 128 * 128;      // 128 rows x 128 bytes
-constexpr int SUB = 64;                    // keys per sub-step
-constexpr int SUB_BYTES = SUB * 128;       // 64 rows of a swizzled half (8 groups of 8 rows x 128 B)
-constexpr int KSTAGES = 2;                 // K ring slots (a third measured neutral)
+constexpr int KSTAGES = 2;                         // K ring slots (a third measured neutral)
 constexpr int VSTAGES = 2;
 constexpr int SQ = 0;                              // Q0 | Q1
 constexpr int SK = SQ + 2 * TILE_BYTES;            // K ring
@@ -56,10 +52,14 @@ constexpr int SBAR = SV + VSTAGES * TILE_BYTES;
 constexpr int SMEM_BYTES = SBAR + 256 + 1024;
 constexpr int THREADS = 384;
 constexpr int REGS_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
-constexpr int REGS_CONTROL = 96;   // warpgroup 0: producer + MMA issuer (88 spills)
-constexpr int REGS_SOFTMAX = 200;  // warpgroups 1, 2
+constexpr int REGS_CONTROL = 88;   // warpgroup 0: producer + MMA issuer
+constexpr int REGS_SOFTMAX = 208;  // warpgroups 1, 2
 static_assert(128 * REGS_CONTROL + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH, "register split");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+// P.V of a key tile goes in two K = 64 halves, the first issued as soon as the
+// softmax has stored the probabilities of keys 0..63 (measured at the 480p
+// shape: two parts ~1210 TFLOP/s, four ~1035, one ~1060).
+constexpr int PV_PARTS = 2;
 }  // namespace attn
 
 __global__ void __launch_bounds__(attn::THREADS, 1)
@@ -74,12 +74,10 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
     uint64_t* k_empty = k_full + KSTAGES;        // [KSTAGES]
     uint64_t* v_full = k_empty + KSTAGES;        // [VSTAGES]
     uint64_t* v_empty = v_full + VSTAGES;        // [VSTAGES]
-    uint64_t* s_full = v_empty + VSTAGES;        // [2 tiles][2 buffers]
-    uint64_t* p_full = s_full + 4;               // [2 tiles][2 buffers] P of a sub-step stored (per buffer:
-                                                 //     the softmax may run two sub-steps ahead of the issuer)
-    uint64_t* pv_done = p_full + 4;              // [2] one completion per P.V of the tile
-    uint64_t* o_final = pv_done + 2;             // [2] the tile's last P.V (pv_done can be two phases
-                                                 //     behind there, so its parity cannot tell)
+    uint64_t* s_full = v_empty + VSTAGES;        // [2] per query tile
+    uint64_t* p_part = s_full + 2;               // [2][PV_PARTS - 1] P columns of the first parts written
+    uint64_t* p_full = p_part + 2 * (PV_PARTS - 1);  // [2]
+    uint64_t* o_final = p_full + 2;              // [2]
     uint64_t* drain = o_final + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -89,7 +87,6 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
     const int h = blockIdx.y, b = blockIdx.z;
     const int q0 = blockIdx.x * 256;
     const int nk = (p.Lk + 127) / 128;
-    const int nsub = (p.Lk + SUB - 1) / SUB;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -101,12 +98,10 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             mbar_init(v_full + s, 1);
             mbar_init(v_empty + s, 1);
         }
-        for (int t = 0; t < 4; ++t) {
-            mbar_init(s_full + t, 1);
-            mbar_init(p_full + t, 4);
-        }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(pv_done + t, 1);
+            mbar_init(s_full + t, 1);
+            for (int q = 0; q < PV_PARTS - 1; ++q) mbar_init(p_part + t * (PV_PARTS - 1) + q, 4);
+            mbar_init(p_full + t, 4);
             mbar_init(o_final + t, 1);
         }
         mbar_init(drain, 1);
@@ -165,7 +160,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
         // warps, so every instruction between MMAs is kept out of the loop:
         // descriptors are built once and moved by adding the offset (>> 4) to
         // their start-address field.
-        constexpr uint32_t ID_QK = idesc_bf16(128, SUB, false);
+        constexpr uint32_t ID_QK = idesc_bf16(128, 128, false);
         constexpr uint32_t ID_PV = idesc_bf16(128, 128, true);
         const uint64_t dq = sdesc_kmajor_sw128(smem_u32(smem + SQ));
         const uint64_t dk = sdesc_kmajor_sw128(smem_u32(smem + SK));
@@ -175,57 +170,65 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             if (lane == 0) r = mbar_wait(bar, parity, abort_flag, p.wc) ? 1 : 0;
             return __shfl_sync(0xffffffffu, r, 0) != 0;
         };
-        // S_t(s) = Q_t K(keys 64 s .. 64 s + 63)^T into buffer s & 1 of tile t
-        auto issue_s = [&](int t, int s) -> bool {
-            const int x = s & 1, j = s >> 1, ks = j % KSTAGES;
-            if (t == 0 && x == 0 && !wait(k_full + ks, (j / KSTAGES) & 1)) return false;
+        bool ok = wait(q_full, 0);
+        // S_t(j) = Q_t K_j^T into TMEM columns [128 t, 128 t + 128)
+        auto issue_s = [&](int t, int j) -> bool {
+            const int ks = j % KSTAGES;
+            if (t == 0 && !wait(k_full + ks, (j / KSTAGES) & 1)) return false;
             tc_fence_after();
             const uint64_t a = dq + (uint64_t)((t * TILE_BYTES) >> 4);
-            const uint64_t bk = dk + (uint64_t)((ks * TILE_BYTES + x * SUB_BYTES) >> 4);
+            const uint64_t b = dk + (uint64_t)((ks * TILE_BYTES) >> 4);
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
-                    umma_bf16_ss(tmem + t * 128 + x * SUB, a + off, bk + off, ID_QK, kk != 0);
+                    umma_bf16_ss(tmem + t * 128, a + off, b + off, ID_QK, kk != 0);
                 }
-                umma_commit(s_full + 2 * t + x);
-                if (t == 1 && (x == 1 || s == nsub - 1)) umma_commit(k_empty + ks);  // last S on this K tile
+                umma_commit(s_full + t);
+                if (t == 1) umma_commit(k_empty + ks);
             }
             __syncwarp();
             issued = true;
             return true;
         };
-        // O_t += P_t(s) V(keys of sub-step s), P_t(s) read from its S columns (bf16 pairs)
-        auto issue_pv = [&](int t, int s) -> bool {
-            const int x = s & 1, j = s >> 1, vs = j % VSTAGES;
-            if (!wait(p_full + 2 * t + x, (s >> 1) & 1)) return false;
-            if (t == 0 && x == 0 && !wait(v_full + vs, (j / VSTAGES) & 1)) return false;
+        // O_t += P_t(j) V_j, P_t read from the S_t columns (bf16 pairs), in
+        // PV_PARTS parts over the keys, each issued as soon as the softmax has
+        // stored its probabilities (p_part), the last after the whole row (p_full)
+        auto issue_pv = [&](int t, int j, int k0, int k1, uint64_t* bar) -> bool {
+            const int vs = j % VSTAGES;
+            const bool last = k1 == 8;
+            if (!wait(bar, j & 1)) return false;
+            if (t == 0 && k0 == 0 && !wait(v_full + vs, (j / VSTAGES) & 1)) return false;
             tc_fence_after();
-            const uint64_t bv = dv + (uint64_t)((vs * TILE_BYTES + x * SUB_BYTES) >> 4);
+            const uint64_t b = dv + (uint64_t)((vs * TILE_BYTES) >> 4);
+            const uint32_t acc0 = (j | k0) != 0;
             if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < SUB / 16; ++kk)
-                    umma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + x * SUB + kk * 8, bv + ((kk * 2048) >> 4),
-                                 ID_PV, (s | kk) != 0);
-                umma_commit(pv_done + t);
-                if (t == 1 && (x == 1 || s == nsub - 1)) umma_commit(v_empty + vs);  // last P.V on this V tile
-                if (s == nsub - 1) umma_commit(o_final + t);
+                for (int kk = k0; kk < k1; ++kk)
+                    umma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b + ((kk * 2048) >> 4), ID_PV,
+                                 kk == k0 ? acc0 : 1u);
+                if (last) {
+                    if (t == 1) umma_commit(v_empty + vs);
+                    if (j == nk - 1) umma_commit(o_final + t);
+                }
             }
             __syncwarp();
             return true;
         };
-        bool ok = wait(q_full, 0);
-        // prologue: both buffers of both tiles (sub-steps 0 and 1)
-#pragma unroll 1
-        for (int i = 0; ok && i < 4 && (i >> 1) < nsub; ++i) ok = issue_s(i & 1, i >> 1);
-        // steady state, per sub-step: PV_0(s) S_0(s+2) PV_1(s) S_1(s+2)
-#pragma unroll 1
-        for (int s = 0; ok && s < nsub; ++s) {
-#pragma unroll 1
-            for (int t = 0; ok && t < 2; ++t) {
-                ok = issue_pv(t, s);
-                if (ok && s + 2 < nsub) ok = issue_s(t, s + 2);
+        auto issue_pv_all = [&](int t, int j) -> bool {
+#pragma unroll
+            for (int q = 0; q < PV_PARTS; ++q) {
+                uint64_t* bar = q == PV_PARTS - 1 ? p_full + t : p_part + t * (PV_PARTS - 1) + q;
+                if (!issue_pv(t, j, q * 8 / PV_PARTS, (q + 1) * 8 / PV_PARTS, bar)) return false;
             }
+            return true;
+        };
+        if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
+        for (int j = 0; ok && j < nk; ++j) {
+            if (!issue_pv_all(0, j)) { ok = false; break; }
+            if (j + 1 < nk && !issue_s(0, j + 1)) { ok = false; break; }
+            if (!issue_pv_all(1, j)) { ok = false; break; }
+            if (j + 1 < nk && !issue_s(1, j + 1)) { ok = false; break; }
         }
     }
     } else {
@@ -235,6 +238,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
         const int qq = warp & 3;                         // TMEM lane quarter
         const int r = qq * 32 + lane;                    // row inside the tile == TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(qq * 32) << 16;
+        const uint32_t TS = tmem + t * 128 + lane_off;   // S_t (and P_t)
         const uint32_t TO = tmem + 256 + t * 128 + lane_off;
         // logits of this thread's query row in log2 units: S * scale_log2, times the
         // row's RMSNorm factor when the queries arrive unnormalised
@@ -250,63 +254,62 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
         }
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
-        for (int s = 0; s < nsub; ++s) {
-            const int x = s & 1;
-            const uint32_t TS = tmem + t * 128 + x * SUB + lane_off;   // S_t(s), then P_t(s)
+        for (int j = 0; j < nk; ++j) {
             // all tcgen05.ld/st below are warp-collective: the warp's decisions stay uniform
-            if (!__all_sync(0xffffffffu, mbar_wait(s_full + 2 * t + x, (s >> 1) & 1, abort_flag, p.wc))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full + t, j & 1, abort_flag, p.wc))) { ok = false; break; }
             tc_fence_after();
-            uint32_t sv[2][32];
-            tmem_ld32(TS, sv[0]);
-            tmem_ld32(TS + 32, sv[1]);
-            tmem_ld_wait(sv[0]);
-            tmem_ld_wait(sv[1]);
-
-            const int valid = min(SUB, p.Lk - s * SUB);
-            if (valid < SUB) {
+            uint32_t sv[4][32];
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < 4; ++c) tmem_ld32(TS + c * 32, sv[c]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
+
+            const int valid = min(128, p.Lk - j * 128);
+            if (valid < 128) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (c * 32 + i >= valid) sv[c][i] = __float_as_uint(-INFINITY);
             }
-            // row maximum: four independent 3-input max chains
-            float mx[4];
+            // row maximum: eight independent 3-input max chains
+            float mx[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 8; ++q) {
                 const uint32_t* v = &sv[q >> 1][(q & 1) * 16];
                 float a = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
 #pragma unroll
                 for (int i = 2; i < 16; i += 2) a = max3f(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
                 mx[q] = a;
             }
-            const float m_tile = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3])) * row_scale;
+            const float m_tile =
+                max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * row_scale;
             const float m_new = fmaxf(m_run, m_tile);
             const bool rescale = m_new > m_run + RESCALE_THRESHOLD;
             const float m_use = rescale ? m_new : m_run;
-            const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;  // 0 on the first sub-step
-            if (s > 0 && __any_sync(0xffffffffu, rescale)) {
-                // O_t must hold every earlier P.V before it is rescaled: wait for P_t(s-1) V
-                if (!__all_sync(0xffffffffu, mbar_wait(pv_done + t, (s - 1) & 1, abort_flag, p.wc))) { ok = false; break; }
-                tc_fence_after();
+            // O_t is idle here (the commit of S_t(j) also covered P_t(j-1) V_{j-1}) and
+            // must be rescaled before the first half of P_t(j) V_j is issued
+            const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;  // 0 on the first tile
+            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {  // 16 columns at a time: the S row stays in registers
-                    uint32_t ov[16];
-                    tmem_ld16(TO + c * 16, ov);
-                    tmem_ld_wait16(ov);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(TO + c * 32, ov);
+                    tmem_ld_wait(ov);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st16(TO + c * 16, ov);
+                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                    tmem_st32(TO + c * 32, ov);
                 }
             }
             // probabilities on packed fp32 pairs, every exponential on the MUFU (scalar
             // FP32 work here would slow the MMA issue on the same sub-partitions);
-            // each 32-column chunk is packed to bf16 and stored over its own S columns
+            // each 32-column chunk is packed to bf16 and stored over its own S
+            // columns (P_t = first 64 columns of S_t) at once
             uint64_t ps2[2] = {0ull, 0ull};
             const uint64_t scale2 = f2pack(row_scale, row_scale);
             const uint64_t negm2 = f2pack(-m_use, -m_use);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 uint32_t pc[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
@@ -318,6 +321,12 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     pc[i / 2] = pack_bf16(e0, e1);
                 }
                 tmem_st16(TS + c * 16, pc);
+                if (c < 3 && (c + 1) % (4 / PV_PARTS) == 0) {  // a part of P (and any O rescale) stored: its P.V may start
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(p_part + t * (PV_PARTS - 1) + (c + 1) / (4 / PV_PARTS) - 1);
+                }
             }
             float ps[4];
             f2unpack(ps2[0], ps[0], ps[1]);
@@ -330,9 +339,8 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full + 2 * t + x);
+            if (lane == 0) mbar_arrive(p_full + t);
         }
-        // the tile's last P.V ends O_t
         if (ok && __all_sync(0xffffffffu, mbar_wait(o_final + t, 0, abort_flag, p.wc))) {
             tc_fence_after();
             const float inv = 1.0f / l_run;

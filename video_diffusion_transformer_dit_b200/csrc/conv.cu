@@ -9,11 +9,12 @@
 // frame 0) and everything else outside the input zero.
 //
 // GEMM view: M = output pixels, N = output channels, K = taps x channels.  A
-// tile is 128 output pixels of one frame (8 rows x 16 columns); for the K
-// block (tap, 64 channels) the producer loads the input patch shifted by the
-// tap with ONE 5-D TMA copy straight from the channels-last input (or the
-// cache), 64 channels x 16 columns x 8 rows = the 128 x 64 K-major tile with
-// 128-byte swizzle the MMA reads.  Zero padding comes free: coordinates
+// tile is 256 output pixels of one frame (16 rows x 16 columns, two 128-row
+// MMA halves sharing each weight tile); for the K block (tap, 64 channels) the
+// producer loads the input patch shifted by the tap with ONE 5-D TMA copy
+// straight from the channels-last input (or the cache), 64 channels x 16
+// columns x 16 rows = two 128 x 64 K-major tiles with 128-byte swizzle, the
+// layout the MMA reads.  Zero padding comes free: coordinates
 // outside the tensor (negative ones included) read as zero.  No im2col matrix
 // is ever written.  The rest is the persistent warp-specialised structure of
 // the linear-layer GEMM: TMA producer warp, single-thread MMA issuer with two
@@ -29,14 +30,15 @@ struct ConvParams {
     int B, T, H, W, Ci, Co;
     int kt, kh, kw, nc;          // kernel; frames in the cache
     int cblocks, kblocks;        // 64-channel blocks per tap; taps * cblocks
-    int ht, wt;                  // spatial tiles of 8 rows x 16 columns
+    int ht, wt;                  // spatial tiles of 16 rows x 16 columns
     int num_m, num_n, num_tiles;
     ConvEpi epi;
     WaitCtl wc;
 };
 
 namespace cv {
-constexpr int BM = 128, BK = 64, TH = 8, TW = 16;
+constexpr int BM = 256, BK = 64, TH = 16, TW = 16;   // 256 pixels = two 128-row MMA halves
+constexpr int HALF_BYTES = 128 * BK * 2;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 template <int BN>
@@ -44,8 +46,10 @@ struct Cfg {
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
-    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int STAGES = (212992 / STAGE_BYTES) < 8 ? (212992 / STAGE_BYTES) : 8;
+    static constexpr int ACC_COLS = 2 * BN;              // both halves of one accumulator set
+    static constexpr int TMEM_COLS = 2 * ACC_COLS;       // double-buffered
+    static_assert(TMEM_COLS <= 512, "tensor memory");
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 };
 }  // namespace cv
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(cv::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * BN;
+                const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
                 for (int kb = 0; kb < p.kblocks; ++kb) {
                     if (!mbar_wait(full + stage, phase, abort_flag, p.wc)) {
                         ok = false;
@@ -218,9 +222,12 @@ __global__ void __launch_bounds__(cv::THREADS, 1)
                     const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
                     const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
-                    for (int k = 0; k < cv::BK / 16; ++k)
-                        umma_bf16_ss(d_tmem, sdesc_kmajor_sw128(a0 + 32 * k), sdesc_kmajor_sw128(b0 + 32 * k), IDESC,
+                    for (int k = 0; k < cv::BK / 16; ++k) {
+                        const uint64_t bd = sdesc_kmajor_sw128(b0 + 32 * k);
+                        umma_bf16_ss(d_tmem, sdesc_kmajor_sw128(a0 + 32 * k), bd, IDESC, (kb | k) != 0);
+                        umma_bf16_ss(d_tmem + BN, sdesc_kmajor_sw128(a0 + cv::HALF_BYTES + 32 * k), bd, IDESC,
                                      (kb | k) != 0);
+                    }
                     issued = true;
                     umma_commit(empty + stage);
                     if (++stage == STAGES) {
@@ -246,16 +253,20 @@ __global__ void __launch_bounds__(cv::THREADS, 1)
             coords(tile, b, t, hb, wb, nb);
             if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc))) break;
             tc_fence_after();
-            const int r = q * 32 + lane;
-            const int h = hb * cv::TH + r / cv::TW, w = wb * cv::TW + r % cv::TW;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
 #pragma unroll 1
-            for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
-                uint32_t rr[32];
-                tmem_ld32(taddr + c0, rr);
-                tmem_ld_wait(rr);
-                const int c = nb * BN + c0;
-                if (h < p.H && w < p.W && c < p.Co) conv_epilogue_chunk(p, b, t, h, w, c, rr);
+            for (int half = 0; half < 2; ++half) {
+                const int r = half * 128 + q * 32 + lane;
+                const int h = hb * cv::TH + r / cv::TW, w = wb * cv::TW + r % cv::TW;
+                const uint32_t taddr =
+                    tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::ACC_COLS + half * BN;
+#pragma unroll 1
+                for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
+                    uint32_t rr[32];
+                    tmem_ld32(taddr + c0, rr);
+                    tmem_ld_wait(rr);
+                    const int c = nb * BN + c0;
+                    if (h < p.H && w < p.W && c < p.Co) conv_epilogue_chunk(p, b, t, h, w, c, rr);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -291,8 +302,7 @@ static cudaError_t conv_attr() {
 }
 
 cudaError_t init_conv_attributes() {
-    cudaError_t e = conv_attr<256>();
-    if (e == cudaSuccess) e = conv_attr<128>();
+    cudaError_t e = conv_attr<128>();
     if (e == cudaSuccess) e = conv_attr<64>();
     return e;
 }
@@ -314,7 +324,7 @@ cudaError_t launch_conv3d(const void* x, const void* cache, int nc, int B, int T
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(cache) |
          reinterpret_cast<uintptr_t>(epi.y) | reinterpret_cast<uintptr_t>(epi.add)) & 15)
         return cudaErrorInvalidValue;
-    const int BN = (Co_pad % 256 == 0) ? 256 : (Co_pad % 128 == 0) ? 128 : 64;
+    const int BN = (Co_pad % 128 == 0) ? 128 : 64;   // two halves x two buffers x BN <= 512 TMEM columns
     ConvParams p{};
     p.B = B; p.T = T; p.H = H; p.W = W; p.Ci = Ci; p.Co = Co;
     p.kt = kt; p.kh = kh; p.kw = kw; p.nc = nc;
@@ -342,11 +352,10 @@ cudaError_t launch_conv3d(const void* x, const void* cache, int nc, int B, int T
     }
     if (!make_tmap_2d(&tw, w, (uint64_t)K, (uint64_t)Co_pad, (uint64_t)ldw, 64, BN)) return cudaErrorInvalidValue;
     const int grid = p.num_tiles < ctx.num_sms ? p.num_tiles : ctx.num_sms;
-    switch (BN) {
-        case 256: conv3d_tc_kernel<256><<<grid, cv::THREADS, cv::Cfg<256>::SMEM_BYTES, ctx.stream>>>(tx, tc, tw, p); break;
-        case 128: conv3d_tc_kernel<128><<<grid, cv::THREADS, cv::Cfg<128>::SMEM_BYTES, ctx.stream>>>(tx, tc, tw, p); break;
-        default: conv3d_tc_kernel<64><<<grid, cv::THREADS, cv::Cfg<64>::SMEM_BYTES, ctx.stream>>>(tx, tc, tw, p); break;
-    }
+    if (BN == 128)
+        conv3d_tc_kernel<128><<<grid, cv::THREADS, cv::Cfg<128>::SMEM_BYTES, ctx.stream>>>(tx, tc, tw, p);
+    else
+        conv3d_tc_kernel<64><<<grid, cv::THREADS, cv::Cfg<64>::SMEM_BYTES, ctx.stream>>>(tx, tc, tw, p);
     if (ctx.launches) ++*ctx.launches;
     return cudaGetLastError();
 }

@@ -314,14 +314,16 @@ __device__ __forceinline__ float epilogue_qk_chunk(const EpiParams& e, int row, 
             v2[2 * i] = mul2(v2[2 * i], g.x);
             v2[2 * i + 1] = mul2(v2[2 * i + 1], g.y);
         }
-        if (e.rope.t) {
+        if (e.rope.t) {  // (pair-major tables) all 16 lookups in flight before any is used
             const int p0 = (c & 127) >> 1;
+            float2 cs[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) cs[i] = __ldg(rope_entry_pm(e.rope, p0 + i, f, ii, jj));
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const float2 cs = rope_cs(e.rope, p0 + i, f, ii, jj);
                 float a, b;
                 f2unpack(v2[i], a, b);
-                v2[i] = fma2(v2[i], f2pack(cs.x, cs.x), mul2(f2pack(b, a), f2pack(-cs.y, cs.y)));
+                v2[i] = fma2(v2[i], f2pack(cs[i].x, cs[i].x), mul2(f2pack(b, a), f2pack(-cs[i].y, cs[i].y)));
             }
         }
     }
@@ -652,8 +654,9 @@ cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long l
         BN = 64;
         if (epi.pair_off < M || !epi.x || !epi.sched || !epi.out) return cudaErrorInvalidValue;
     }
-    if (epi.kind == EPI_QK_NORM) {
-        if (N % 256 || epi.norm_cols < 0 || epi.norm_cols % 128 || epi.norm_cols > N || !epi.ssq ||
+    if (epi.kind == EPI_QK_NORM) {  // the epilogue reads pair-major RoPE tables
+        if ((epi.rope.t && !epi.rope.pair_major) ||
+            N % 256 || epi.norm_cols < 0 || epi.norm_cols % 128 || epi.norm_cols > N || !epi.ssq ||
             (epi.norm_cols > 0 && !epi.gain) || epi.ssq_ld < epi.norm_cols / 128 || epi.ldo % 8 ||
             (epi.rope.t && epi.rope_L <= 0))
             return cudaErrorInvalidValue;

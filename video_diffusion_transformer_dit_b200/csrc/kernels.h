@@ -135,6 +135,14 @@ __device__ __forceinline__ float2 rope_cs(const RopeTables& rt, int p, int f, in
     p -= rt.nh;
     return __ldg(rt.w + j * rt.nw + p);
 }
+// Address of the (cos, sin) entry of pair p in pair-major tables, without
+// branches (selects), so that a run of lookups can all be in flight at once.
+__device__ __forceinline__ const float2* rope_entry_pm(const RopeTables& rt, int p, int f, int i, int j) {
+    const float2* at_t = rt.t + p * rt.Fp + f;
+    const float2* at_h = rt.h + (p - rt.nt) * rt.Hp + i;
+    const float2* at_w = rt.w + (p - rt.nt - rt.nh) * rt.Wp + j;
+    return p < rt.nt ? at_t : (p < rt.nt + rt.nh ? at_h : at_w);
+}
 #endif
 
 // Row widths and strides the RMSNorm kernels take: D a supported multiple of

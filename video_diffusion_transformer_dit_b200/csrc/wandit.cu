@@ -133,6 +133,12 @@ struct wan_dit {
     bool sp_active = false;
     int sp_B = 0, sp_F = 0, sp_Hz = 0, sp_Wz = 0, sp_Lc = 0, sp_per_token = 0, sp_dtype = 0;
     int sp_rank = 0, sp_world = 0, sp_Ls = 0;
+    // whole latent in and whole velocity out of a sequence-parallel forward (the
+    // workspace holds only the shard's tokens); allocated by the first sp_begin of a size
+    void* sp_lat = nullptr;
+    size_t sp_lat_bytes = 0;
+    float* sp_vel = nullptr;
+    size_t sp_vel_bytes = 0;
     int sp_next_block = 0;
     int sp_phase = 0;     // 0: next call is sp_block_qkv, 1: sp_block_finish
 };
@@ -442,8 +448,8 @@ cudaError_t issue_prologue(wan_dit* h, const Shape& s, const LaunchCtx& ctx, boo
     const int B = s.B, Lr = s.rows_per_sample(), Lc = s.Lc, D = c.dim, N = c.num_blocks;
     const int R = B * Lr, Rc = B * Lc;
     const long long D6 = 6LL * D;
-    TRYK(WAN_KC_PATCHIFY, wan::launch_patchify(h->lat_stage, s.lat_dtype, B, c.in_ch, s.F, s.Hz, s.Wz, h->X, h->Kp, ctx,
-                                               s.world ? s.tok0 : 0, Lr));
+    TRYK(WAN_KC_PATCHIFY, wan::launch_patchify(s.world ? h->sp_lat : h->lat_stage, s.lat_dtype, B, c.in_ch, s.F, s.Hz,
+                                               s.Wz, h->X, h->Kp, ctx, s.world ? s.tok0 : 0, Lr));
     TRYK(WAN_KC_GEMM, wan::launch_gemm(h->X, h->Kp, h->w_pe_k, h->Kp, R, D, h->Kp,
                                        make_epi(wan::EPI_BIAS, h->b_pe, h->x, D), ctx));
     if (dump) TRY(cudaMemcpyAsync(h->dump, h->x, (size_t)R * D * 2, cudaMemcpyDeviceToDevice, ctx.stream));
@@ -589,7 +595,8 @@ cudaError_t issue_head(wan_dit* h, const Shape& s, const LaunchCtx& ctx, KTimer*
     const int R = B * Lr;
     TRYK(WAN_KC_LAYERNORM, wan::launch_layernorm(h->x, h->y, R, D, c.eps, 0, nullptr, nullptr, h->sst_out, h->temb,
                                                  h->sst_out + D, h->temb, s.per_token ? 1 : Lr, D, ctx));
-    EpiParams p = make_epi(s.cfg_euler ? wan::EPI_CFG_EULER : wan::EPI_UNPATCHIFY, h->b_po, h->vel_stage, 0);
+    EpiParams p = make_epi(s.cfg_euler ? wan::EPI_CFG_EULER : wan::EPI_UNPATCHIFY, h->b_po,
+                           s.world ? h->sp_vel : h->vel_stage, 0);
     p.L = L;
     p.C = c.out_ch;
     p.F = s.F;
@@ -745,6 +752,8 @@ void wan_dit_destroy(wan_dit* h) {
     if (h->arena) cudaFree(h->arena);
     if (h->ws) cudaFree(h->ws);
     if (h->d_err) cudaFree(h->d_err);
+    if (h->sp_lat) cudaFree(h->sp_lat);
+    if (h->sp_vel) cudaFree(h->sp_vel);
     delete h;
 }
 
@@ -1062,7 +1071,22 @@ wan_status wan_dit_sp_begin(wan_dit* h, const void* latent, int latent_dtype, in
     if (ps != WAN_OK) return ps;
     const cudaMemcpyKind h2d = io_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
     const size_t lat_bytes = (size_t)B * c.in_ch * F * Hz * Wz * (latent_dtype == WAN_DTYPE_F32 ? 4 : 2);
-    WAN_CU(cudaMemcpyAsync(h->lat_stage, latent, lat_bytes, h2d, st), "latent copy");
+    const size_t vel_bytes = (size_t)B * c.out_ch * F * Hz * Wz * 4;
+    if (lat_bytes > h->sp_lat_bytes) {
+        if (h->sp_lat) cudaFree(h->sp_lat);
+        h->sp_lat = nullptr;
+        h->sp_lat_bytes = 0;
+        WAN_CU(cudaMalloc(&h->sp_lat, lat_bytes), "sequence-parallel latent staging");
+        h->sp_lat_bytes = lat_bytes;
+    }
+    if (vel_bytes > h->sp_vel_bytes) {
+        if (h->sp_vel) cudaFree(h->sp_vel);
+        h->sp_vel = nullptr;
+        h->sp_vel_bytes = 0;
+        WAN_CU(cudaMalloc(&h->sp_vel, vel_bytes), "sequence-parallel velocity staging");
+        h->sp_vel_bytes = vel_bytes;
+    }
+    WAN_CU(cudaMemcpyAsync(h->sp_lat, latent, lat_bytes, h2d, st), "latent copy");
     if (per_token) {  // this shard's columns of the [B, L] timesteps; padding tokens get t = 0
         const long long tok0 = (long long)rank * Ls, n = std::max(0LL, std::min(Ls, L - tok0));
         WAN_CU(cudaMemsetAsync(h->t_stage, 0, (size_t)B * Ls * 4, st), "timestep clear");
@@ -1145,11 +1169,11 @@ wan_status wan_dit_sp_end(wan_dit* h, float* velocity, int io_on_device, void* s
     const Shape s = sp_shape(h);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t vel_bytes = (size_t)s.B * h->cfg.out_ch * s.F * s.Hz * s.Wz * 4;
-    WAN_CU(cudaMemsetAsync(h->vel_stage, 0, vel_bytes, st), "velocity clear");
+    WAN_CU(cudaMemsetAsync(h->sp_vel, 0, vel_bytes, st), "velocity clear");
     LaunchCtx ctx = make_ctx(h, st, nullptr);
     cudaError_t e = issue_head(h, s, ctx, nullptr);
     if (e != cudaSuccess) return cuda_fail(h, e, "sequence-parallel head");
-    WAN_CU(cudaMemcpyAsync(velocity, h->vel_stage, vel_bytes, io_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+    WAN_CU(cudaMemcpyAsync(velocity, h->sp_vel, vel_bytes, io_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
                            st),
            "velocity copy");
     h->sp_active = false;
