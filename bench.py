@@ -194,7 +194,7 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from video_diffusion_transformer_dit_b200 import build, configs, synth
-    from video_diffusion_transformer_dit_b200.binding import WAN_OPT_KERNEL_TIMING, WanDiT
+    from video_diffusion_transformer_dit_b200.binding import WAN_OPT_GEMM_PAIR, WAN_OPT_KERNEL_TIMING, WanDiT
 
     build.build()
     torch.cuda.set_device(local_rank)
@@ -220,6 +220,7 @@ def run_ours(args, rank, world, local_rank):
     img = synth.make_image(B, Li, cfg["image_dim"], seed=args.seed, device=str(dev)) if Li else None
     dit = WanDiT(cfg, max_batch=B, max_tokens=L, max_text=Lc, device=local_rank, max_image=max(Li, 1))
     dit.load_weights(W)
+    dit.set_option(WAN_OPT_GEMM_PAIR, args.gemm_pair)
     del W
     torch.cuda.synchronize()
     vel = torch.empty(B, cfg["out_ch"], F, Hz, Wz, device=dev)
@@ -306,7 +307,8 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic latents/contexts, random-init bf16 weights of the named shapes",
-        "config": dict(arm_config(args.workload, world), **({"blocks": args.blocks} if args.blocks else {})),
+        "config": dict(arm_config(args.workload, world), **({"blocks": args.blocks} if args.blocks else {}),
+                       **({} if args.gemm_pair else {"gemm_pair": 0})),
         "tflops_per_step": flops / 1e12,
         "achieved_tflops": flops / (ms * 1e-3) / 1e12,
         "tc_peak_frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
@@ -333,7 +335,8 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------- single-kernel mode
-KERNELS = ("self_attention", "cross_attention", "gemm_qkv", "gemm_o", "gemm_ffn_up", "gemm_ffn_down", "layernorm",
+KERNELS = ("self_attention", "cross_attention", "gemm_qkv", "gemm_qkv_norm", "gemm_o", "gemm_ffn_up", "gemm_ffn_down",
+           "layernorm",
            "rmsnorm_rope", "vae_conv", "vae_decode")
 
 
@@ -394,6 +397,7 @@ def run_kernel(args):
     from video_diffusion_transformer_dit_b200 import binding as Bd
     from video_diffusion_transformer_dit_b200 import build, configs
     build.build()
+    Bd.op_set_gemm_pair(bool(args.gemm_pair))
     w = configs.workload(args.workload)
     cfg = w["cfg"]
     B, Cc, F, Hz, Wz = w["latent"]
@@ -421,7 +425,8 @@ def run_kernel(args):
                                              o.data_ptr(), D, B, H, L, Lk)
         work, unit = 4.0 * L * Lk * D * B, "TFLOP/s"
     elif k.startswith("gemm"):
-        N, K_, epi = {"gemm_qkv": (3 * D, D, "bias"), "gemm_o": (D, D, "gate_residual"),
+        N, K_, epi = {"gemm_qkv": (3 * D, D, "bias"), "gemm_qkv_norm": (3 * D, D, "bias"),
+                      "gemm_o": (D, D, "gate_residual"),
                       "gemm_ffn_up": (Fd, D, "bias_gelu"), "gemm_ffn_down": (D, Fd, "gate_residual")}[k]
         A = rnd(R, K_)
         Wt = rnd(N, K_, scale=0.02)
@@ -430,6 +435,11 @@ def run_kernel(args):
         gate0 = torch.full((N,), 0.1, device=dev)
         gate1 = torch.zeros(B, 6 * N, device=dev)
         fn = lambda: Bd.op_gemm(A, Wt, epi, out, bias=bias, gate0=gate0, gate1=gate1, mod_div=L, mod_ld=6 * N)
+        if k == "gemm_qkv_norm":   # q/k gain, RoPE and per-head sums of squares in the epilogue
+            gain = torch.ones(2 * D, device=dev)
+            ssq = torch.empty(R, 2 * H, device=dev)
+            fn = lambda: Bd.op_gemm(A, Wt, "qk_norm", out, bias=bias, gain=gain, ssq=ssq, norm_cols=2 * D,
+                                    rope_grid=(F, Hz // 2, Wz // 2))
         work, unit = 2.0 * R * N * K_, "TFLOP/s"
     elif k == "layernorm":
         x = rnd(R, D)
@@ -480,6 +490,8 @@ def main():
                          "in config.blocks; not a measurement of the named model)")
     ap.add_argument("--kernel", choices=KERNELS, default=None,
                     help="time one kernel alone at the workload's shapes (profiling aid)")
+    ap.add_argument("--gemm-pair", type=int, choices=[0, 1], default=1,
+                    help="1: GEMMs with N a multiple of 256 on SM pairs (default); 0: single-SM tiles only")
     args = ap.parse_args()
     if args.kernel in ("vae_conv", "vae_decode"):
         return run_vae(args)

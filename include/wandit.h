@@ -254,8 +254,12 @@ WANDIT_API wan_status wan_dit_set_block_dump(wan_dit* h, void* dst);
  * default 1), WAN_OPT_WAIT_LIMIT_NS (time limit of every on-chip wait,
  * default 2e9 ns; values below 1000 are for fault tests only),
  * WAN_OPT_KERNEL_TIMING (1 = record a CUDA event pair around every kernel of
- * the forward, read back with wan_dit_kernel_time; default 0).            */
-enum { WAN_OPT_GRAPH = 1, WAN_OPT_WAIT_LIMIT_NS = 2, WAN_OPT_KERNEL_TIMING = 3 };
+ * the forward, read back with wan_dit_kernel_time; default 0),
+ * WAN_OPT_GEMM_PAIR (1 = the block GEMMs with N a multiple of 256 run as
+ * SM-pair tcgen05 GEMMs, 256 x 256 tiles on clusters of two CTAs; 0 = every
+ * GEMM on single-SM 128-row tiles; default 1; same results either way up to
+ * fp32 summation order).                                                   */
+enum { WAN_OPT_GRAPH = 1, WAN_OPT_WAIT_LIMIT_NS = 2, WAN_OPT_KERNEL_TIMING = 3, WAN_OPT_GEMM_PAIR = 4 };
 
 /* Kernel classes of the forward, for wan_dit_kernel_time().  WAN_KC_GEMM
  * covers the GEMMs outside the blocks (patch, timestep, text, cross K/V,

@@ -208,6 +208,17 @@ WANDIT_API wan_status wan_op_sync(void* stream);
 /* Time limit in ns of every on-chip wait of the op kernels (default 2e9). */
 WANDIT_API void wan_op_set_wait_limit_ns(int64_t ns);
 
+/* wan_op_gemm on SM pairs where it applies (on != 0, the default: N a
+ * multiple of 256, M >= 512, bias / GELU / gate-residual / residual / q-k
+ * norm epilogues) or always on single-SM tiles (on == 0).                  */
+WANDIT_API void wan_op_set_gemm_pair(int on);
+
+/* Number of two-CTA clusters the SM-pair GEMM runs with on the current
+ * device (0 if the device cannot co-schedule them; the GEMMs then use
+ * single-SM tiles).  Initialises the op state of the device; -1 on a CUDA
+ * error.                                                                   */
+WANDIT_API int wan_op_gemm_pair_clusters(void);
+
 #ifdef __cplusplus
 }
 #endif

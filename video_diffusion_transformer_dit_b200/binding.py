@@ -19,7 +19,7 @@ WAN_STATUS = {0: "WAN_OK", 1: "WAN_EINVAL", 2: "WAN_ESHAPE", 3: "WAN_ENOMEM", 4:
               5: "WAN_EMISSING_WEIGHT", 6: "WAN_EUNEXPECTED_WEIGHT", 7: "WAN_ECUDA", 8: "WAN_ETIMEOUT",
               9: "WAN_EINTERNAL", 10: "WAN_EUNSUPPORTED"}
 WAN_DTYPE_F32, WAN_DTYPE_BF16 = 0, 1
-WAN_OPT_GRAPH, WAN_OPT_WAIT_LIMIT_NS, WAN_OPT_KERNEL_TIMING = 1, 2, 3
+WAN_OPT_GRAPH, WAN_OPT_WAIT_LIMIT_NS, WAN_OPT_KERNEL_TIMING, WAN_OPT_GEMM_PAIR = 1, 2, 3, 4
 KERNEL_CLASSES = {"patchify": 0, "gemm": 1, "self_attention": 2, "cross_attention": 3, "layernorm": 4,
                   "rmsnorm_rope": 5, "embedding": 6, "gemm_qkv": 7, "gemm_o": 8, "gemm_q2": 9, "gemm_o2": 10,
                   "gemm_ffn_up": 11, "gemm_ffn_down": 12}
@@ -37,7 +37,7 @@ SYMBOLS = ["wan_dit_create", "wan_dit_load_weights", "wan_dit_missing_weights", 
            "wan_op_attention_qnorm", "wan_op_rms_apply", "wan_dit_sp_begin", "wan_dit_sp_block_qkv",
            "wan_dit_sp_attention", "wan_dit_sp_block_finish", "wan_dit_sp_end",
            "wan_vae_create", "wan_vae_load_weights", "wan_vae_missing_weights", "wan_vae_decode", "wan_vae_sync",
-           "wan_vae_last_error", "wan_vae_destroy", "wan_op_conv3d"]
+           "wan_vae_last_error", "wan_vae_destroy", "wan_op_conv3d", "wan_op_set_gemm_pair", "wan_op_gemm_pair_clusters"]
 
 
 class WanError(RuntimeError):
@@ -107,6 +107,8 @@ def lib() -> C.CDLL:
         "wan_op_wait_selftest": (I, [I64, P]),
         "wan_op_causal_conv3d": (I, [P, P, I, I, I, I, I, I, P, I64, P, I, I, I, I, P, I64, P, P]),
         "wan_op_set_wait_limit_ns": (None, [I64]),
+        "wan_op_set_gemm_pair": (None, [I]),
+        "wan_op_gemm_pair_clusters": (I, []),
         "wan_dit_forward_cfg_euler": (I, [P, P, I, I, I, F, P, I, F, F, F, P, I, P]),
         "wan_flow_sigmas": (I, [I, D, C.POINTER(D)]),
         "wan_op_attention_qnorm": (I, [P, I64, P, I64, P, I64, P, I64, I, I, I, I, P, I64, I, F, P]),
@@ -506,3 +508,16 @@ def op_sync(stream=None):
 
 def op_set_wait_limit_ns(ns: int):
     lib().wan_op_set_wait_limit_ns(int(ns))
+
+
+def op_set_gemm_pair(on: bool):
+    """op_gemm on SM-pair (cta_group::2) tiles where it applies, or always single-SM."""
+    lib().wan_op_set_gemm_pair(1 if on else 0)
+
+
+def op_gemm_pair_clusters() -> int:
+    """Two-CTA clusters the SM-pair GEMM runs with on this device (0: unavailable)."""
+    n = lib().wan_op_gemm_pair_clusters()
+    if n < 0:
+        raise WanError(7, "wan_op_gemm_pair_clusters")
+    return n

@@ -369,6 +369,52 @@ __device__ __forceinline__ void epilogue_cfg_euler(const EpiParams& e, int row, 
     }
 }
 
+// One epilogue warp's share of an accumulator tile: TMEM lanes of its quarter
+// (rows `row`), columns [chalf * BN/2, (chalf + 1) * BN/2) of tile column `nb`.
+template <int BN, int KIND, bool PAIR>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, int row, int nb, uint32_t taddr, int chalf) {
+    constexpr int CW = BN / 2;  // columns per epilogue warp
+    if constexpr (KIND == EPI_QK_NORM) {
+        // this warp's 128 columns are one head: its sum of squares is one ssq entry
+        static_assert(BN == 256, "one 128-column group per epilogue warp");
+        const int gcol = nb * BN + chalf * CW;
+        const bool normed = gcol < p.epi.norm_cols;
+        int f = 0, ii = 0, jj = 0;
+        if (normed && p.epi.rope.t) {
+            const int hw = p.epi.rope.Hp * p.epi.rope.Wp;
+            const int l = min(p.epi.rope_tok0 + row % p.epi.rope_L, p.epi.rope.Fp * hw - 1);
+            f = l / hw;
+            const int rem = l - f * hw;
+            ii = rem / p.epi.rope.Wp;
+            jj = rem - ii * p.epi.rope.Wp;
+        }
+        float ss = 0.0f;
+#pragma unroll 1
+        for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c0, r);
+            tmem_ld_wait(r);
+            if (row < p.M) ss += epilogue_qk_chunk(p.epi, row, nb * BN + c0, r, normed, f, ii, jj);
+        }
+        if (normed && row < p.M) p.epi.ssq[(long long)row * p.epi.ssq_ld + gcol / 128] = ss;
+    } else {
+#pragma unroll 1
+        for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c0, r);
+            tmem_ld_wait(r);
+            if constexpr (PAIR) {
+                uint32_t ru[32];
+                tmem_ld32(taddr + BN + c0, ru);
+                tmem_ld_wait(ru);
+                if (row < p.M) epilogue_cfg_euler(p.epi, row, nb * BN + c0, r, ru);
+            } else {
+                if (row < p.M) epilogue_chunk<KIND>(p.epi, row, nb * BN + c0, r);
+            }
+        }
+    }
+}
+
 constexpr int EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
 
@@ -502,7 +548,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // ---------------- epilogue warps ----------------
         const int q = warp & 3;                       // TMEM lane quarter this warp may access
         const int chalf = (warp - 2) >> 2;            // which half of the tile's columns
-        constexpr int CW = BN / 2;                    // columns per epilogue warp
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
@@ -513,44 +558,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tc_fence_after();
             const int row = mb * 128 + q * 32 + lane;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * (Cfg::NA * BN);
-            if constexpr (KIND == EPI_QK_NORM) {
-                // this warp's 128 columns are one head: its sum of squares is one ssq entry
-                static_assert(BN == 256, "one 128-column group per epilogue warp");
-                const int gcol = nb * BN + chalf * CW;
-                const bool normed = gcol < p.epi.norm_cols;
-                int f = 0, ii = 0, jj = 0;
-                if (normed && p.epi.rope.t) {
-                    const int hw = p.epi.rope.Hp * p.epi.rope.Wp;
-                    const int l = min(p.epi.rope_tok0 + row % p.epi.rope_L, p.epi.rope.Fp * hw - 1);
-                    f = l / hw;
-                    const int rem = l - f * hw;
-                    ii = rem / p.epi.rope.Wp;
-                    jj = rem - ii * p.epi.rope.Wp;
-                }
-                float ss = 0.0f;
-#pragma unroll 1
-                for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(taddr + c0, r);
-                    tmem_ld_wait(r);
-                    if (row < p.M) ss += epilogue_qk_chunk(p.epi, row, nb * BN + c0, r, normed, f, ii, jj);
-                }
-                if (normed && row < p.M) p.epi.ssq[(long long)row * p.epi.ssq_ld + gcol / 128] = ss;
-            } else
-#pragma unroll 1
-            for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(taddr + c0, r);
-                tmem_ld_wait(r);
-                if constexpr (PAIR) {
-                    uint32_t ru[32];
-                    tmem_ld32(taddr + BN + c0, ru);
-                    tmem_ld_wait(ru);
-                    if (row < p.M) epilogue_cfg_euler(p.epi, row, nb * BN + c0, r, ru);
-                } else {
-                    if (row < p.M) epilogue_chunk<KIND>(p.epi, row, nb * BN + c0, r);
-                }
-            }
+            epilogue_tile<BN, KIND, PAIR>(p, row, nb, taddr, chalf);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + acc);
@@ -578,6 +586,231 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
 }
 
+// ----------------------------------------------------------------------------
+// SM-pair GEMM (tcgen05 .cta_group::2): a cluster of two CTAs computes a
+// 256 x 256 tile; the even CTA issues one M = 256, N = 256, K = 16 MMA per
+// 16-deep K slice.  Each CTA stages its own 128 A rows and its own 128-row half
+// of the W tile (32 KB per 64-deep K step instead of the 48 KB a 128 x 256
+// single-SM tile needs), and the tensor cores of the pair read both halves of
+// W, which halves W's shared-memory and L2 traffic per SM.  Each CTA's tensor
+// memory holds the accumulator rows of its own A rows (all 256 columns), so
+// the epilogue is the single-SM one.
+//
+// Barriers sit at the same shared-memory offsets in both CTAs:
+//   full[s]    even CTA: 1 arrival (its producer, announcing the bytes of both
+//              CTAs' loads) + those bytes, which each CTA's loads deliver;
+//   empty[s]   both: 1 arrival, the MMA commit multicast to the pair;
+//   tfull[a]   both: 1 arrival, the MMA commit multicast to the pair;
+//   tempty[a]  even CTA: 16 arrivals, the 8 epilogue warps of each CTA.
+// All handshakes use CTA-scope acquire / release, also across the pair: the
+// data they guard moves through the async proxy (TMA bytes counted on the
+// barrier, MMA commits) or through tensor memory under tcgen05 fences, and a
+// cluster-scope release would put a memory barrier into every K step.
+// Teardown: both CTAs stop issuing, synchronise, and if either gave up a wait
+// the even CTA completes every full[s] phase a load of either CTA went into
+// and drains its MMAs before the pair synchronises again and frees its
+// tensor memory.
+// ----------------------------------------------------------------------------
+namespace pair2 {
+constexpr int BN = 256;
+constexpr int HALF_BYTES = 128 * 64 * 2;      // one 128 x 64 bf16 operand tile
+constexpr int STAGE_BYTES = 2 * HALF_BYTES;   // A rows + W half
+constexpr int STAGES = 6;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+// loads a producer that issued n loads put into stage s
+__device__ __forceinline__ uint32_t loads_in_stage(uint32_t n, int s) {
+    return n > (uint32_t)s ? (n - 1 - s) / STAGES + 1 : 0u;
+}
+}  // namespace pair2
+
+template <int KIND>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+    gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmParams p) {
+    using namespace pair2;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;                          // [STAGES] this CTA's 128 A rows x 64
+    uint8_t* sB = smem + STAGES * HALF_BYTES;    // [STAGES] this CTA's 128 W rows x 64
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile uint32_t* loads_issued = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();     // 0: the CTA that issues the MMAs
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull + a, 1);
+            mbar_init(tempty + a, 2 * EPI_WARPS);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        *loads_issued = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();   // barriers initialised and tensor memory allocated in both CTAs
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int kblocks = p.K / 64;
+    const int cid = static_cast<int>(cluster_id_x());
+    const int ncl = static_cast<int>(num_clusters_x());
+    uint32_t n_loads = 0;
+    bool issued = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs) ----------------
+            const uint32_t full0 = mapa_shared(smem_u32(full), 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = cid; ok && tile < p.num_tiles; tile += ncl) {
+                int mb, nb;
+                tile_coords(tile, p, mb, nb);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.wc)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = full0 + 8u * stage;
+                    if (leader) mbar_expect_tx(full + stage, 2 * STAGE_BYTES);
+                    tma_load_2d_pair(sA + stage * HALF_BYTES, &tmA, fb, kb * 64, mb * 256 + rank * 128);
+                    tma_load_2d_pair(sB + stage * HALF_BYTES, &tmB, fb, kb * 64, nb * BN + rank * 128);
+                    ++n_loads;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // the MMA commits that free this CTA's stages arrive here: wait for
+            // the last of them so none lands after the CTA has exited
+            for (int s = 0; ok && s < STAGES; ++s) {
+                const uint32_t c = loads_in_stage(n_loads, s);
+                if (c) ok = mbar_wait(empty + s, (c - 1) & 1u, abort_flag, p.wc);
+            }
+            *loads_issued = n_loads;
+        }
+    } else if (warp == 1) {
+        if (leader && lane == 0) {
+            // ---------------- MMA issuer (even CTA) ----------------
+            constexpr uint32_t IDESC = idesc_bf16(256, BN, false);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = cid; ok && tile < p.num_tiles; tile += ncl) {
+                if (!mbar_wait(tempty + acc, acc_phase ^ 1, abort_flag, p.wc)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(full + stage, phase, abort_flag, p.wc)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * HALF_BYTES);
+                    const uint32_t b0 = smem_u32(sB + stage * HALF_BYTES);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_bf16_ss_pair(d_tmem, sdesc_kmajor_sw128(a0 + 32 * k), sdesc_kmajor_sw128(b0 + 32 * k),
+                                          IDESC, (kb | k) != 0);
+                    issued = true;
+                    umma_commit_pair_mc(empty + stage, 0x3);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                umma_commit_pair_mc(tfull + acc, 0x3);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+        }
+    } else {
+        // ---------------- epilogue warps (both CTAs) ----------------
+        const int q = warp & 3;
+        const int chalf = (warp - 2) >> 2;
+        const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = cid; tile < p.num_tiles; tile += ncl) {
+            int mb, nb;
+            tile_coords(tile, p, mb, nb);
+            if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc))) break;
+            tc_fence_after();
+            const int row = mb * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+            epilogue_tile<BN, KIND, false>(p, row, nb, taddr, chalf);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(tempty0 + 8u * acc);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+
+    __syncthreads();
+    cluster_sync_all();   // neither CTA issues another load, MMA or arrival
+    const bool any_abort =
+        *abort_flag != 0 || ld_shared_cluster_u32(mapa_shared(smem_u32((const void*)abort_flag), rank ^ 1u)) != 0;
+    if (any_abort && leader && lane == 0) {
+        if (warp == 0) {
+            // every full[s] phase that a load of either CTA went into completes
+            // once the loads issued into it have landed.  The two producers'
+            // counts per stage differ by at most one (a load of phase j waits
+            // for phase j - 1 to be consumed); where the odd CTA stopped first,
+            // its bytes are counted as delivered, where the even CTA did, the
+            // arrival it owed is made for the odd CTA's bytes alone
+            const uint32_t n0 = *loads_issued;
+            const uint32_t n1 = ld_shared_cluster_u32(mapa_shared(smem_u32((const void*)loads_issued), 1));
+            for (int s = 0; s < STAGES; ++s) {
+                const uint32_t c0 = loads_in_stage(n0, s), c1 = loads_in_stage(n1, s);
+                const uint32_t c = c0 > c1 ? c0 : c1;
+                if (!c) continue;
+                if (c0 > c1) mbar_complete_tx(full + s, STAGE_BYTES);
+                if (c1 > c0) mbar_expect_tx(full + s, STAGE_BYTES);
+                mbar_drain(full + s, (c - 1) & 1u, 200000000ull);
+            }
+        } else if (warp == 1 && issued) {
+            umma_commit_pair(drain);
+            mbar_drain(drain, 0, 200000000ull);
+        }
+    }
+    __syncthreads();
+    cluster_sync_all();   // the pair's loads and MMAs have landed
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 template <int BN, int KIND>
 static cudaError_t set_gemm_attr_one() {
     return cudaFuncSetAttribute(gemm_tc_kernel<BN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -596,8 +829,44 @@ static cudaError_t set_gemm_attr() {
     return e;
 }
 
+// Clusters of two that fit on the device at once with one pair CTA per SM
+// (0: the pair kernel is not used).
+static int g_pair_clusters = 0;
+
+template <int KIND>
+static cudaError_t set_pair_attr_one() {
+    return cudaFuncSetAttribute(gemm_pair_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                pair2::SMEM_BYTES);
+}
+
+static cudaError_t init_pair_gemm() {
+    cudaError_t e = set_pair_attr_one<EPI_BIAS>();
+    if (e == cudaSuccess) e = set_pair_attr_one<EPI_BIAS_GELU>();
+    if (e == cudaSuccess) e = set_pair_attr_one<EPI_GATE_RESIDUAL>();
+    if (e == cudaSuccess) e = set_pair_attr_one<EPI_RESIDUAL>();
+    if (e == cudaSuccess) e = set_pair_attr_one<EPI_QK_NORM>();
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = pair2::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_tc_kernel<EPI_BIAS>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    g_pair_clusters = n;
+    return cudaSuccess;
+}
+
+int gemm_pair_clusters() { return g_pair_clusters; }
+
 cudaError_t init_gemm_attributes() {
-    cudaError_t e = set_gemm_attr<256>();
+    cudaError_t e = init_pair_gemm();
+    if (e == cudaSuccess) e = set_gemm_attr<256>();
     if (e == cudaSuccess) e = set_gemm_attr<128>();
     if (e == cudaSuccess) e = set_gemm_attr<64>();
     if (e == cudaSuccess) e = set_gemm_attr_one<64, EPI_CFG_EULER>();
@@ -661,11 +930,14 @@ cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long l
             (epi.rope.t && epi.rope_L <= 0))
             return cudaErrorInvalidValue;
     }
+    const bool use_pair = ctx.gemm_pair && g_pair_clusters > 0 && BN == 256 && M >= 512 &&
+                          (epi.kind == EPI_BIAS || epi.kind == EPI_BIAS_GELU || epi.kind == EPI_GATE_RESIDUAL ||
+                           epi.kind == EPI_RESIDUAL || epi.kind == EPI_QK_NORM);
     GemmParams p;
     p.M = M;
     p.N = N;
     p.K = K;
-    p.num_m = (M + 127) / 128;
+    p.num_m = use_pair ? (M + 255) / 256 : (M + 127) / 128;
     p.num_n = N / BN;
     p.num_tiles = p.num_m * p.num_n;
     // walk M fastest when the weight operand is the bigger one (few row blocks)
@@ -678,7 +950,26 @@ cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long l
     // the pair variant reads the second sample's rows [pair_off, pair_off + M) as well
     const uint64_t a_rows = pair ? (uint64_t)epi.pair_off + (uint64_t)M : (uint64_t)M;
     if (!make_tmap_2d(&ta, A, K, a_rows, lda, 64, 128)) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&tb, W, K, N, ldw, 64, BN)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tb, W, K, N, ldw, 64, use_pair ? 128 : BN)) return cudaErrorInvalidValue;
+    if (use_pair) {
+        const int clusters = p.num_tiles < g_pair_clusters ? p.num_tiles : g_pair_clusters;
+        switch (epi.kind) {
+#define WAN_PAIR_CASE(K)                                                                                 \
+    case K:                                                                                              \
+        gemm_pair_tc_kernel<K><<<2 * clusters, GEMM_THREADS, pair2::SMEM_BYTES, ctx.stream>>>(ta, tb, p); \
+        break;
+            WAN_PAIR_CASE(EPI_BIAS)
+            WAN_PAIR_CASE(EPI_BIAS_GELU)
+            WAN_PAIR_CASE(EPI_GATE_RESIDUAL)
+            WAN_PAIR_CASE(EPI_RESIDUAL)
+            WAN_PAIR_CASE(EPI_QK_NORM)
+#undef WAN_PAIR_CASE
+            default:
+                return cudaErrorInvalidValue;
+        }
+        if (ctx.launches) ++*ctx.launches;
+        return cudaGetLastError();
+    }
     switch (BN) {
         case 256: return launch_gemm_bn<256>(ta, tb, p, ctx);
         case 128: return launch_gemm_bn<128>(ta, tb, p, ctx);

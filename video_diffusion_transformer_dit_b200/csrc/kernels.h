@@ -70,6 +70,7 @@ struct LaunchCtx {
     uint64_t wait_limit_ns;
     int num_sms;
     int* launches;          // incremented per kernel launch (host counter), may be null
+    int gemm_pair = 1;      // 1: large N % 256 == 0 GEMMs run on SM pairs (cta_group::2)
 };
 
 // Raise the dynamic shared-memory limit of the tcgen05 kernels (once per
@@ -87,6 +88,9 @@ bool make_tmap_5d(CUtensorMap* m, const void* ptr, const uint64_t (&dims)[5], co
 
 // C = epi(A[M,K] . W[N,K]^T); returns a CUDA error (or cudaErrorInvalidValue
 // for unsupported shapes).
+// Two-CTA clusters the SM-pair GEMM runs with (0: not available); valid after
+// init_kernel_attributes().
+int gemm_pair_clusters();
 cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long ldw, int M, int N, int K,
                         const EpiParams& epi, const LaunchCtx& ctx);
 

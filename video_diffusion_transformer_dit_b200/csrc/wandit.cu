@@ -127,6 +127,7 @@ struct wan_dit {
     cudaStream_t cap_stream = nullptr;
     std::map<PlanKey, Plan> plans;
     bool timing = false;
+    bool gemm_pair = true;
     Plan* last_plan = nullptr;
     bool last_timed = false;
     // sequence-parallel forward in progress (between wan_dit_sp_begin and wan_dit_sp_end)
@@ -676,6 +677,7 @@ LaunchCtx make_ctx(wan_dit* h, cudaStream_t st, int* counter) {
     ctx.wait_limit_ns = h->wait_ns;
     ctx.num_sms = h->num_sms;
     ctx.launches = counter;
+    ctx.gemm_pair = h->gemm_pair ? 1 : 0;
     return ctx;
 }
 
@@ -866,6 +868,15 @@ wan_status wan_dit_set_option(wan_dit* h, int option, int64_t value) {
     }
     if (option == WAN_OPT_KERNEL_TIMING) {
         h->timing = value != 0;
+        return WAN_OK;
+    }
+    if (option == WAN_OPT_GEMM_PAIR) {
+        h->gemm_pair = value != 0;
+        for (auto& kv : h->plans) {  // graphs hold the old kernels
+            if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+            if (kv.second.exec_timed) cudaGraphExecDestroy(kv.second.exec_timed);
+            kv.second.exec = kv.second.exec_timed = nullptr;
+        }
         return WAN_OK;
     }
     return fail(h, WAN_EINVAL, "unknown option");
@@ -1228,6 +1239,7 @@ struct OpState {
     int* d_err = nullptr;
     int num_sms = 148;
     uint64_t wait_ns = kDefaultWaitNs;
+    int gemm_pair = 1;
 };
 std::mutex g_op_mu;
 std::map<int, OpState> g_ops;
@@ -1249,6 +1261,7 @@ bool op_ctx(cudaStream_t st, LaunchCtx* ctx) {
     ctx->wait_limit_ns = s.wait_ns;
     ctx->num_sms = s.num_sms;
     ctx->launches = nullptr;
+    ctx->gemm_pair = s.gemm_pair;
     return true;
 }
 
@@ -1264,6 +1277,19 @@ void wan_op_set_wait_limit_ns(int64_t ns) {
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lk(g_op_mu);
     g_ops[dev].wait_ns = ns < 0 ? 0 : (uint64_t)ns;
+}
+
+void wan_op_set_gemm_pair(int on) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_op_mu);
+    g_ops[dev].gemm_pair = on ? 1 : 0;
+}
+
+int wan_op_gemm_pair_clusters(void) {
+    LaunchCtx ctx;
+    if (!op_ctx(nullptr, &ctx)) return -1;
+    return wan::gemm_pair_clusters();
 }
 
 wan_status wan_op_sync(void* stream) {
