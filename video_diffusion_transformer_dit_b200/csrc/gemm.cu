@@ -59,8 +59,16 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmParams& p, int& 
 // pairs; bias, GELU, gate and residual run as f32x2 operations, which keeps
 // the scalar FP32 pipe free for the MMA-issuing warp on the same SM
 // sub-partitions (scalar FFMA traffic there slows tcgen05.mma issue).
+// Residual rows of one 32-column chunk (4 x 16 B), loaded ahead of their use.
+__device__ __forceinline__ void load_residual(const EpiParams& e, int row, int c, uint4 (&xu)[4]) {
+    const uint4* xp = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xu[i] = xp[i];
+}
+
 template <int KIND>
-__device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, int c, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, int c, const uint32_t (&r)[32],
+                                                  const uint4 (&xu)[4]) {
     uint64_t v2[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) v2[i] = f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
@@ -90,38 +98,30 @@ __device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, i
             }
             dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-    } else {  // EPI_GATE_RESIDUAL, EPI_RESIDUAL
-        // issue every load of the chunk before any store: x (4 x 16 B) and the gate rows
+    } else {  // EPI_GATE_RESIDUAL, EPI_RESIDUAL: x (4 x 16 B) arrives preloaded
         uint4* xp = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
-        uint4 xu[4];
+        const ulonglong2* g1 =
+            e.gate1 ? reinterpret_cast<const ulonglong2*>(e.gate1 + (long long)(row / e.mod_div) * e.mod_ld + c) : nullptr;
+        const ulonglong2* g0 = e.gate0 ? reinterpret_cast<const ulonglong2*>(e.gate0 + c) : nullptr;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) xu[i] = xp[i];
-        uint64_t g2[16];
-        if (KIND == EPI_GATE_RESIDUAL) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) g2[i] = 0ull;  // +0.0f, +0.0f
-            if (e.gate1) {
-                const ulonglong2* g =
-                    reinterpret_cast<const ulonglong2*>(e.gate1 + (long long)(row / e.mod_div) * e.mod_ld + c);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const ulonglong2 a = __ldg(g + i);
-                    g2[2 * i] = a.x;
-                    g2[2 * i + 1] = a.y;
+        for (int i = 0; i < 4; ++i) {  // 8 columns: 16 B of x, 4 pairs of the gate
+            uint64_t g2[4] = {0ull, 0ull, 0ull, 0ull};  // +0.0f pairs
+            if (KIND == EPI_GATE_RESIDUAL) {
+                if (g1) {
+                    const ulonglong2 a0 = __ldg(g1 + 2 * i), a1 = __ldg(g1 + 2 * i + 1);
+                    g2[0] = a0.x;
+                    g2[1] = a0.y;
+                    g2[2] = a1.x;
+                    g2[3] = a1.y;
+                }
+                if (g0) {
+                    const ulonglong2 a0 = __ldg(g0 + 2 * i), a1 = __ldg(g0 + 2 * i + 1);
+                    g2[0] = add2(g2[0], a0.x);
+                    g2[1] = add2(g2[1], a0.y);
+                    g2[2] = add2(g2[2], a1.x);
+                    g2[3] = add2(g2[3], a1.y);
                 }
             }
-            if (e.gate0) {
-                const ulonglong2* g = reinterpret_cast<const ulonglong2*>(e.gate0 + c);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const ulonglong2 a = __ldg(g + i);
-                    g2[2 * i] = add2(g2[2 * i], a.x);
-                    g2[2 * i + 1] = add2(g2[2 * i + 1], a.y);
-                }
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
             const uint32_t xw[4] = {xu[i].x, xu[i].y, xu[i].z, xu[i].w};
             uint32_t ow[4];
 #pragma unroll
@@ -130,7 +130,7 @@ __device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, i
                 const uint64_t x2 = f2pack(xf.x, xf.y);
                 uint64_t o2;
                 if (KIND == EPI_GATE_RESIDUAL) {
-                    o2 = fma2(v2[4 * i + h], g2[4 * i + h], x2);
+                    o2 = fma2(v2[4 * i + h], g2[h], x2);
                 } else {  // the branch output is rounded to bf16 before the residual add
                     float a, b;
                     f2unpack(v2[4 * i + h], a, b);
@@ -149,8 +149,9 @@ __device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, i
 // Epilogue of 32 consecutive columns [c, c + 32) of one row (KIND fixed at compile time).
 template <int KIND>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int c, const uint32_t (&r)[32]) {
-    if constexpr (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU || KIND == EPI_GATE_RESIDUAL || KIND == EPI_RESIDUAL) {
-        epilogue_chunk_f2<KIND>(e, row, c, r);
+    if constexpr (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU) {
+        const uint4 none[4] = {};
+        epilogue_chunk_f2<KIND>(e, row, c, r, none);
     } else {
     float v[32];
 #pragma unroll
@@ -369,12 +370,41 @@ __device__ __forceinline__ void epilogue_cfg_euler(const EpiParams& e, int row, 
     }
 }
 
+__host__ __device__ constexpr bool reads_residual(int kind) { return kind == EPI_GATE_RESIDUAL || kind == EPI_RESIDUAL; }
+
+// Residual of the first chunk of an epilogue warp's share of tile (row, nb),
+// loaded before the warp waits for the accumulator.
+template <int BN, int KIND>
+__device__ __forceinline__ void epilogue_prefetch(const GemmParams& p, int row, int nb, int chalf, uint4 (&x0)[4]) {
+    if constexpr (reads_residual(KIND)) {
+        if (row < p.M) load_residual(p.epi, row, nb * BN + chalf * (BN / 2), x0);
+    }
+}
+
 // One epilogue warp's share of an accumulator tile: TMEM lanes of its quarter
 // (rows `row`), columns [chalf * BN/2, (chalf + 1) * BN/2) of tile column `nb`.
+// x0: the residual of its first chunk (residual epilogues).
 template <int BN, int KIND, bool PAIR>
-__device__ __forceinline__ void epilogue_tile(const GemmParams& p, int row, int nb, uint32_t taddr, int chalf) {
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, int row, int nb, uint32_t taddr, int chalf,
+                                              uint4 (&x0)[4]) {
     constexpr int CW = BN / 2;  // columns per epilogue warp
-    if constexpr (KIND == EPI_QK_NORM) {
+    if constexpr (reads_residual(KIND)) {
+        // the residual of chunk k + 1 loads while chunk k is computed, through
+        // two buffers (a buffer is reused only after its values are consumed)
+        uint4 x1[4];
+        auto chunk = [&](int k, uint4 (&use)[4], uint4 (&next)[4]) {
+            const int c0 = chalf * CW + k * 32;
+            if (k + 1 < CW / 32 && row < p.M) load_residual(p.epi, row, nb * BN + c0 + 32, next);
+            uint32_t r[32];
+            tmem_ld32(taddr + c0, r);
+            tmem_ld_wait(r);
+            if (row < p.M) epilogue_chunk_f2<KIND>(p.epi, row, nb * BN + c0, r, use);
+        };
+        chunk(0, x0, x1);
+        if constexpr (CW / 32 > 1) chunk(1, x1, x0);
+        if constexpr (CW / 32 > 2) chunk(2, x0, x1);
+        if constexpr (CW / 32 > 3) chunk(3, x1, x0);
+    } else if constexpr (KIND == EPI_QK_NORM) {
         // this warp's 128 columns are one head: its sum of squares is one ssq entry
         static_assert(BN == 256, "one 128-column group per epilogue warp");
         const int gcol = nb * BN + chalf * CW;
@@ -553,12 +583,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
             int mb, nb;
             tile_coords(tile, p, mb, nb);
+            const int row = mb * 128 + q * 32 + lane;
+            uint4 x0[4];
+            epilogue_prefetch<BN, KIND>(p, row, nb, chalf, x0);
             // tcgen05.ld is warp-collective: the whole warp takes the same branch
             if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc))) break;
             tc_fence_after();
-            const int row = mb * 128 + q * 32 + lane;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * (Cfg::NA * BN);
-            epilogue_tile<BN, KIND, PAIR>(p, row, nb, taddr, chalf);
+            epilogue_tile<BN, KIND, PAIR>(p, row, nb, taddr, chalf, x0);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + acc);
@@ -762,11 +794,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         for (int tile = cid; tile < p.num_tiles; tile += ncl) {
             int mb, nb;
             tile_coords(tile, p, mb, nb);
+            const int row = mb * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+            uint4 x0[4];
+            epilogue_prefetch<BN, KIND>(p, row, nb, chalf, x0);
             if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc))) break;
             tc_fence_after();
-            const int row = mb * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-            epilogue_tile<BN, KIND, false>(p, row, nb, taddr, chalf);
+            epilogue_tile<BN, KIND, false>(p, row, nb, taddr, chalf, x0);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(tempty0 + 8u * acc);
