@@ -444,10 +444,10 @@ def run_kernel(args):
     elif k == "layernorm":
         x = rnd(R, D)
         y = torch.empty_like(x)
-        sst = torch.zeros(6, D, device=dev)
         tp = torch.zeros(B, 6 * D, device=dev)
-        fn = lambda: Bd.op_layernorm(x, y, 1e-6, 0, shift0=sst[0], shift1=tp, scale0=sst[1], scale1=tp,
-                                     mod_div=L, mod_ld=6 * D)
+        # mode 2, the block LayerNorms: per-sample scale (1 + scale included) and shift rows
+        fn = lambda: Bd.op_layernorm(x, y, 1e-6, 2, shift1=tp[:, 0:D], scale1=tp[:, D:2 * D], mod_div=L,
+                                     mod_ld=6 * D)
         work, unit = 2.0 * R * D * 2, "GB/s"
     elif k == "rmsnorm_rope":
         qkv = rnd(R, 3 * D)

@@ -111,7 +111,11 @@ WANDIT_API wan_status wan_op_rms_apply(void* buf, int64_t ld, int rows, int D, c
 /* LayerNorm of bf16 rows x[rows, D] (fp32 statistics, biased variance, eps),
  * then either an affine (gamma, beta; mode 1: norm2) or the adaLN modulation
  * (mode 0: y = LN(x) * (1 + scale0[c] + scale1[m c]) + shift0[c] + shift1[m c],
- * m = r / mod_div, row stride mod_ld; norm1/norm3/norm_out).  Output bf16.  */
+ * m = r / mod_div, row stride mod_ld; norm_out), or the modulation with the
+ * per-sample rows already combined (mode 2: y = LN(x) * scale1[m c] +
+ * shift1[m c], scale1 holding 1 + scale; the forward's norm1/norm3, whose
+ * rows come from the all-blocks modulation table).  D a multiple of 256;
+ * WAN_EINVAL for another mode or a missing vector.  Output bf16.            */
 WANDIT_API wan_status wan_op_layernorm(const void* x, void* y, int rows, int D, float eps, int mode,
                             const float* gamma, const float* beta,
                             const float* shift0, const float* shift1,

@@ -247,6 +247,35 @@ def test_layernorm_affine():
     assert rel_l2(y, O.layer_norm(x.to(DT), 1e-6, gam.to(DT), bet.to(DT))) < TOL
 
 
+@pytest.mark.parametrize("D", [256, 1536])
+def test_layernorm_row_walking_modes(D):
+    """Enough rows (>= 8 warps per SM) for the kernel in which each warp walks
+    consecutive rows with the modulation in registers: mode 2 (precombined
+    per-sample scale / shift, the sample boundary 2123 falls inside a warp's
+    rows) and mode 1 (affine); 4246 rows leave the last warp a ragged share."""
+    rows, L = 4246, 2123
+    g = torch.Generator().manual_seed(70 + D)
+    x = (torch.randn(rows, D, generator=g) * 2 + 0.5).to(torch.bfloat16)
+    scale1 = 1 + torch.randn(2, D, generator=g) * 0.2
+    shift1 = torch.randn(2, D, generator=g) * 0.2
+    tab = torch.zeros(2, 6 * D)
+    tab[:, 0:D], tab[:, D:2 * D] = shift1, scale1
+    tab = tab.cuda()
+    y = torch.full((rows, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    B().op_layernorm(x.cuda(), y, 1e-6, 2, shift1=tab[:, 0:D], scale1=tab[:, D:2 * D], mod_div=L, mod_ld=6 * D)
+    B().op_sync()
+    ln = O.layer_norm(x.to(DT), 1e-6)
+    ref = ln * scale1.to(DT).repeat_interleave(L, 0) + shift1.to(DT).repeat_interleave(L, 0)
+    assert not torch.isnan(y.float()).any()
+    assert rel_l2(y, ref) < TOL
+    gam, bet = scale1[0].contiguous(), shift1[1].contiguous()
+    y.fill_(float("nan"))
+    B().op_layernorm(x.cuda(), y, 1e-6, 1, gamma=gam.cuda(), beta=bet.cuda())
+    B().op_sync()
+    assert not torch.isnan(y.float()).any()
+    assert rel_l2(y, O.layer_norm(x.to(DT), 1e-6, gam.to(DT), bet.to(DT))) < TOL
+
+
 @pytest.mark.parametrize("rope", [False, True])
 def test_rmsnorm_rope(rope):
     Fp, Hp, Wp = 3, 5, 7

@@ -100,6 +100,98 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __r
     }
 }
 
+// LayerNorm modes 1 and 2 for D <= 1536, each warp walking `rpw` consecutive rows
+// (a grid of one 256-thread CTA per SM).  The warp's columns of the
+// modulation (or affine) vectors stay in registers and are reloaded only when
+// the rows cross into the next sample, so per row only x and y move through
+// L1 (the per-row reload of 8 bytes of fp32 vectors per element made the
+// one-row-per-warp kernel L1-bound); rows are loaded two ahead of their use.
+template <int NCH, int MODE>
+__global__ void __launch_bounds__(256, 1)
+    layernorm_rows_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y, int rows, int rpw,
+                          float eps, const float* gamma, const float* beta, const float* shift0, const float* shift1,
+                          const float* scale0, const float* scale1, int mod_div, long long mod_ld) {
+    constexpr int D = NCH * 256;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = (blockIdx.x * 8 + warp) * rpw;
+    const int r1 = min(r0 + rpw, rows);
+    if (r0 >= r1) return;
+    float ga[NCH][8], gb[NCH][8];  // y = (x - mean) * rstd * ga + gb on this lane's columns
+    long long m_cur = -1;
+    auto load_mod = [&](long long m) {
+#pragma unroll
+        for (int t = 0; t < NCH; ++t) {
+            const int c = (t * 32 + lane) * 8;
+            if (MODE == 2) {
+                load8f(scale1 + m + c, ga[t]);
+                load8f(shift1 + m + c, gb[t]);
+            } else {
+                load8f(gamma + c, ga[t]);
+                load8f(beta + c, gb[t]);
+            }
+        }
+    };
+    auto load_row = [&](int row, uint4 (&u)[NCH]) {
+        if (row < r1) {
+            const __nv_bfloat16* xr = x + (long long)row * D;
+#pragma unroll
+            for (int t = 0; t < NCH; ++t) u[t] = *reinterpret_cast<const uint4*>(xr + (t * 32 + lane) * 8);
+        }
+    };
+    auto do_row = [&](int row, const uint4 (&u)[NCH]) {
+        if (row >= r1) return;
+        if (MODE != 1) {
+            const long long m = (long long)(row / mod_div) * mod_ld;
+            if (m != m_cur) {
+                load_mod(m);
+                m_cur = m;
+            }
+        }
+        float s = 0.f;
+#pragma unroll
+        for (int t = 0; t < NCH; ++t) {
+            float v[8];
+            unpack8(u[t], v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s += v[i];
+        }
+        const float mean = warp_sum(s) * (1.0f / D);
+        float ss = 0.f;
+#pragma unroll
+        for (int t = 0; t < NCH; ++t) {
+            float v[8];
+            unpack8(u[t], v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float d = v[i] - mean;
+                ss += d * d;
+            }
+        }
+        const float rstd = rsqrtf(warp_sum(ss) * (1.0f / D) + eps);
+        __nv_bfloat16* yr = y + (long long)row * D;
+#pragma unroll
+        for (int t = 0; t < NCH; ++t) {
+            float v[8], o[8];
+            unpack8(u[t], v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = (v[i] - mean) * rstd * ga[t][i] + gb[t][i];
+            store8(yr + (t * 32 + lane) * 8, o);
+        }
+    };
+    if (MODE == 1) load_mod(0);
+    uint4 ua[NCH], ub[NCH], uc[NCH];
+    load_row(r0, ua);
+    load_row(r0 + 1, ub);
+    for (int row = r0; row < r1; row += 3) {  // three buffers: each is refilled right after its row is done
+        load_row(row + 2, uc);
+        do_row(row, ua);
+        load_row(row + 3, ua);
+        do_row(row + 1, ub);
+        load_row(row + 4, ub);
+        do_row(row + 2, uc);
+    }
+}
+
 cudaError_t launch_layernorm(const void* x, void* y, int rows, int D, float eps, int mode, const float* gamma,
                              const float* beta, const float* shift0, const float* shift1, const float* scale0,
                              const float* scale1, int mod_div, long long mod_ld, const LaunchCtx& ctx) {
@@ -109,6 +201,29 @@ cudaError_t launch_layernorm(const void* x, void* y, int rows, int D, float eps,
     dim3 grid((rows + 7) / 8);
     auto X = reinterpret_cast<const __nv_bfloat16*>(x);
     auto Y = reinterpret_cast<__nv_bfloat16*>(y);
+    // rows walked per warp, modulation kept in registers (modes 1 and 2: mode 0
+    // needs the vectors of two sources combined and would spill)
+    if (D <= 1536 && mode != 0 && rows >= 8 * ctx.num_sms) {
+        const int warps = 8 * ctx.num_sms;
+        const int rpw = (rows + warps - 1) / warps;
+        const int blocks = (rows + 8 * rpw - 1) / (8 * rpw);
+#define WAN_LN_ROWS(n)                                                                                          \
+    case n:                                                                                                     \
+        if (mode == 2)                                                                                          \
+            layernorm_rows_kernel<n, 2><<<blocks, 256, 0, ctx.stream>>>(X, Y, rows, rpw, eps, gamma, beta, shift0, \
+                                                                        shift1, scale0, scale1, mod_div, mod_ld); \
+        else                                                                                                    \
+            layernorm_rows_kernel<n, 1><<<blocks, 256, 0, ctx.stream>>>(X, Y, rows, rpw, eps, gamma, beta, shift0, \
+                                                                        shift1, scale0, scale1, mod_div, mod_ld); \
+        break;
+        switch (D / 256) {
+            WAN_LN_ROWS(1) WAN_LN_ROWS(2) WAN_LN_ROWS(3) WAN_LN_ROWS(4) WAN_LN_ROWS(6)
+            default: return cudaErrorInvalidValue;
+        }
+#undef WAN_LN_ROWS
+        if (ctx.launches) ++*ctx.launches;
+        return cudaGetLastError();
+    }
 #define WAN_LN_CASE(n)                                                                                             \
     case n:                                                                                                        \
         if (mode == 2)                                                                                             \

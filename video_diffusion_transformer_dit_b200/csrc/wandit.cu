@@ -1413,7 +1413,8 @@ wan_status wan_op_layernorm(const void* x, void* y, int rows, int D, float eps, 
     if (!x || !y) return WAN_EINVAL;
     if (mode == 0 && (!shift0 || !shift1 || !scale0 || !scale1)) return WAN_EINVAL;
     if (mode == 1 && (!gamma || !beta)) return WAN_EINVAL;
-    if (mode != 0 && mode != 1) return WAN_EINVAL;
+    if (mode == 2 && (!shift1 || !scale1)) return WAN_EINVAL;
+    if (mode != 0 && mode != 1 && mode != 2) return WAN_EINVAL;
     LaunchCtx ctx;
     if (!op_ctx(reinterpret_cast<cudaStream_t>(stream), &ctx)) return WAN_ECUDA;
     return op_status(
