@@ -186,6 +186,34 @@ def test_attention(Bn, heads, Lq, Lk):
     assert rel_l2(o, ref) < TOL
 
 
+@pytest.mark.parametrize("Lk", [226, 300, 512])
+def test_attention_units_walked_per_cta(Lk):
+    """Short key sets (2, 3 or 4 key tiles) run with one CTA per SM walking
+    256-query units; B = 2, 12 heads, Lq = 2000 (eight query blocks, the last
+    ragged) give 192 units, so CTAs take one or two units and the barrier
+    phases carry over between them; compared with the oracle per element and
+    against a run whose units fit one per CTA (the first two heads alone)."""
+    Bn, heads, Lq = 2, 12, 2000
+    D = heads * 128
+    g = torch.Generator().manual_seed(90 + Lk)
+    q = torch.randn(Bn * Lq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(Bn * Lk, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(Bn * Lk, D, generator=g).to(torch.bfloat16)
+    o = torch.full((Bn * Lq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    B().op_attention(q.cuda(), k.cuda(), v.cuda(), o, Bn, heads, Lq, Lk)
+    B().op_sync()
+    ref = O.attention(q.to(DT).reshape(Bn, Lq, heads, 128), k.to(DT).reshape(Bn, Lk, heads, 128),
+                      v.to(DT).reshape(Bn, Lk, heads, 128)).reshape(Bn * Lq, D)
+    assert not torch.isnan(o.float()).any()
+    assert rel_l2(o, ref) < TOL
+    # two heads: 32 units, one per CTA; same per-row arithmetic, same bits
+    o2 = torch.empty(Bn * Lq, 256, dtype=torch.bfloat16, device="cuda")
+    B().op_attention(q[:, :256].contiguous().cuda(), k[:, :256].contiguous().cuda(), v[:, :256].contiguous().cuda(),
+                     o2, Bn, 2, Lq, Lk)
+    B().op_sync()
+    assert torch.equal(o2.cpu(), o.cpu()[:, :256])
+
+
 def test_attention_strided_qkv_buffer():
     """q, k, v as column slices of one [rows, 3D] buffer, as the forward uses them."""
     Bn, heads, L = 2, 2, 260

@@ -3,10 +3,17 @@
 // Used for the self-attention over the L video tokens and the
 // cross-attention to the Lc text tokens (ragged key tail masked).
 //
-// One CTA per (256 queries = two 128-row tiles, head, batch), 12 warps in
+// Work unit: 256 queries (two 128-row tiles) of one (head, batch).  A CTA
+// walks units blockIdx.x, blockIdx.x + gridDim.x, ...: one unit per CTA for
+// the self-attention (grid = units), one CTA per SM for short key sets such
+// as the cross-attention's text tokens, where a unit is only a few key tiles
+// and the set-up (barriers, tensor memory, the first Q load) would otherwise
+// be paid per unit.  Barrier phases run on over the units: Q once per unit
+// (the next unit's Q loads as soon as the last S MMA of the current one has
+// read Q), K / V / S / P once per key tile.  12 warps in
 // three warpgroups; the first gives registers to the two softmax groups
-// (88 / 208 / 208 per thread, 64512 in all = 384 threads x 168 at launch):
-//   warp 0      TMA producer: both Q tiles once, then K and V tiles of 128
+// (96 / 200 / 200 per thread, 63488 of the 384 x 168 = 64512 at launch):
+//   warp 0      TMA producer: both Q tiles of a unit, then K and V tiles of 128
 //               keys in two-slot rings (3-D tensor maps: rows past the
 //               sequence read as zero);
 //   warp 1      tensor-memory owner and MMA issuer.  Tensor memory holds
@@ -33,6 +40,7 @@ namespace wan {
 
 struct AttnParams {
     int Lq, Lk, heads;
+    int nqb, units;    // 256-row query blocks per (head, batch); nqb * heads * batch
     __nv_bfloat16* o;
     long long ldo;
     float scale_log2;  // log2(e) / sqrt(head_dim)
@@ -52,8 +60,8 @@ constexpr int SBAR = SV + VSTAGES * TILE_BYTES;
 constexpr int SMEM_BYTES = SBAR + 256 + 1024;
 constexpr int THREADS = 384;
 constexpr int REGS_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
-constexpr int REGS_CONTROL = 88;   // warpgroup 0: producer + MMA issuer
-constexpr int REGS_SOFTMAX = 208;  // warpgroups 1, 2
+constexpr int REGS_CONTROL = 96;   // warpgroup 0: producer + MMA issuer
+constexpr int REGS_SOFTMAX = 200;  // warpgroups 1, 2
 static_assert(128 * REGS_CONTROL + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH, "register split");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 // P.V of a key tile goes in two K = 64 halves, the first issued as soon as the
@@ -70,7 +78,8 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SBAR);
     uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;                 // [KSTAGES]
+    uint64_t* q_empty = bars + 1;                // every S MMA of the unit has read Q
+    uint64_t* k_full = bars + 2;                 // [KSTAGES]
     uint64_t* k_empty = k_full + KSTAGES;        // [KSTAGES]
     uint64_t* v_full = k_empty + KSTAGES;        // [VSTAGES]
     uint64_t* v_empty = v_full + VSTAGES;        // [VSTAGES]
@@ -84,12 +93,18 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int h = blockIdx.y, b = blockIdx.z;
-    const int q0 = blockIdx.x * 256;
     const int nk = (p.Lk + 127) / 128;
+    // unit u -> (query block, head, batch), query blocks fastest
+    auto coords = [&](int u, int& q0, int& h, int& b) {
+        q0 = (u % p.nqb) * 256;
+        const int r = u / p.nqb;
+        h = r % p.heads;
+        b = r / p.heads;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int s = 0; s < KSTAGES; ++s) {
             mbar_init(k_full + s, 1);
             mbar_init(k_empty + s, 1);
@@ -119,9 +134,11 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // producer: ring slots with a load issued and the phase it completes; MMA
-    // issuer: whether any MMA went out (both drained after an abort, before exit)
+    // producer: ring slots with a load issued and the phase it completes, and the
+    // phase of the last Q load; MMA issuer: whether any MMA went out (both
+    // drained after an abort, before exit)
     uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
+    int qpar = -1;
     bool issued = false;
 
     if (warp < 4) {
@@ -130,14 +147,20 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
         if (lane == 0) {
             // ---------------- producer ----------------
             bool ok = true;
+            int g = 0;  // key tiles loaded so far, over all units of this CTA
+            for (int u = blockIdx.x, i = 0; ok && u < p.units; u += gridDim.x, ++i) {
+            int q0, h, b;
+            coords(u, q0, h, b);
+            if (!mbar_wait(q_empty, (i & 1) ^ 1, abort_flag, p.wc)) { ok = false; break; }
             mbar_expect_tx(q_full, 2 * TILE_BYTES);
             for (int t = 0; t < 2; ++t) {
                 tma_load_3d(smem + SQ + t * TILE_BYTES, &tmQ, q_full, h * 128, q0 + 128 * t, b);
                 tma_load_3d(smem + SQ + t * TILE_BYTES + HALF_BYTES, &tmQ, q_full, h * 128 + 64, q0 + 128 * t, b);
             }
-            for (int j = 0; ok && j < nk; ++j) {
-                const int ks = j % KSTAGES, vs = j % VSTAGES;
-                const uint32_t kp = (j / KSTAGES) & 1, vp = (j / VSTAGES) & 1;
+            qpar = i & 1;
+            for (int j = 0; ok && j < nk; ++j, ++g) {
+                const int ks = g % KSTAGES, vs = g % VSTAGES;
+                const uint32_t kp = (g / KSTAGES) & 1, vp = (g / VSTAGES) & 1;
                 if (!mbar_wait(k_empty + ks, kp ^ 1, abort_flag, p.wc)) { ok = false; break; }
                 mbar_expect_tx(k_full + ks, TILE_BYTES);
                 tma_load_3d(smem + SK + ks * TILE_BYTES, &tmK, k_full + ks, h * 128, j * 128, b);
@@ -150,6 +173,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                 tma_load_3d(smem + SV + vs * TILE_BYTES + HALF_BYTES, &tmV, v_full + vs, h * 128 + 64, j * 128, b);
                 varmed |= 1u << vs;
                 vpar = (vpar & ~(1u << vs)) | (vp << vs);
+            }
             }
         }
     } else if (warp == 1) {
@@ -170,11 +194,12 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             if (lane == 0) r = mbar_wait(bar, parity, abort_flag, p.wc) ? 1 : 0;
             return __shfl_sync(0xffffffffu, r, 0) != 0;
         };
-        bool ok = wait(q_full, 0);
-        // S_t(j) = Q_t K_j^T into TMEM columns [128 t, 128 t + 128)
-        auto issue_s = [&](int t, int j) -> bool {
-            const int ks = j % KSTAGES;
-            if (t == 0 && !wait(k_full + ks, (j / KSTAGES) & 1)) return false;
+        // S_t(j) = Q_t K_j^T into TMEM columns [128 t, 128 t + 128); gj counts key
+        // tiles over all units (ring slots and phases), the unit's last S also
+        // releases Q for the next unit
+        auto issue_s = [&](int t, int gj, bool last) -> bool {
+            const int ks = gj % KSTAGES;
+            if (t == 0 && !wait(k_full + ks, (gj / KSTAGES) & 1)) return false;
             tc_fence_after();
             const uint64_t a = dq + (uint64_t)((t * TILE_BYTES) >> 4);
             const uint64_t b = dk + (uint64_t)((ks * TILE_BYTES) >> 4);
@@ -186,6 +211,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                 }
                 umma_commit(s_full + t);
                 if (t == 1) umma_commit(k_empty + ks);
+                if (t == 1 && last) umma_commit(q_empty);
             }
             __syncwarp();
             issued = true;
@@ -194,11 +220,12 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
         // O_t += P_t(j) V_j, P_t read from the S_t columns (bf16 pairs), in
         // PV_PARTS parts over the keys, each issued as soon as the softmax has
         // stored its probabilities (p_part), the last after the whole row (p_full)
-        auto issue_pv = [&](int t, int j, int k0, int k1, uint64_t* bar) -> bool {
-            const int vs = j % VSTAGES;
+        // (j: the key tile inside the unit, gj: over all units)
+        auto issue_pv = [&](int t, int gj, int j, int k0, int k1, uint64_t* bar) -> bool {
+            const int vs = gj % VSTAGES;
             const bool last = k1 == 8;
-            if (!wait(bar, j & 1)) return false;
-            if (t == 0 && k0 == 0 && !wait(v_full + vs, (j / VSTAGES) & 1)) return false;
+            if (!wait(bar, gj & 1)) return false;
+            if (t == 0 && k0 == 0 && !wait(v_full + vs, (gj / VSTAGES) & 1)) return false;
             tc_fence_after();
             const uint64_t b = dv + (uint64_t)((vs * TILE_BYTES) >> 4);
             const uint32_t acc0 = (j | k0) != 0;
@@ -215,20 +242,24 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             __syncwarp();
             return true;
         };
-        auto issue_pv_all = [&](int t, int j) -> bool {
+        auto issue_pv_all = [&](int t, int gj, int j) -> bool {
 #pragma unroll
             for (int q = 0; q < PV_PARTS; ++q) {
                 uint64_t* bar = q == PV_PARTS - 1 ? p_full + t : p_part + t * (PV_PARTS - 1) + q;
-                if (!issue_pv(t, j, q * 8 / PV_PARTS, (q + 1) * 8 / PV_PARTS, bar)) return false;
+                if (!issue_pv(t, gj, j, q * 8 / PV_PARTS, (q + 1) * 8 / PV_PARTS, bar)) return false;
             }
             return true;
         };
-        if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
-        for (int j = 0; ok && j < nk; ++j) {
-            if (!issue_pv_all(0, j)) { ok = false; break; }
-            if (j + 1 < nk && !issue_s(0, j + 1)) { ok = false; break; }
-            if (!issue_pv_all(1, j)) { ok = false; break; }
-            if (j + 1 < nk && !issue_s(1, j + 1)) { ok = false; break; }
+        bool ok = true;
+        int g = 0;  // first key tile of the unit, counted over all units
+        for (int u = blockIdx.x, i = 0; ok && u < p.units; u += gridDim.x, ++i, g += nk) {
+            ok = wait(q_full, i & 1) && issue_s(0, g, nk == 1) && issue_s(1, g, nk == 1);
+            for (int j = 0; ok && j < nk; ++j) {
+                if (!issue_pv_all(0, g + j, j)) { ok = false; break; }
+                if (j + 1 < nk && !issue_s(0, g + j + 1, j + 2 == nk)) { ok = false; break; }
+                if (!issue_pv_all(1, g + j, j)) { ok = false; break; }
+                if (j + 1 < nk && !issue_s(1, g + j + 1, j + 2 == nk)) { ok = false; break; }
+            }
         }
     }
     } else {
@@ -240,23 +271,27 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
         const uint32_t lane_off = static_cast<uint32_t>(qq * 32) << 16;
         const uint32_t TS = tmem + t * 128 + lane_off;   // S_t (and P_t)
         const uint32_t TO = tmem + 256 + t * 128 + lane_off;
+        bool ok = true;
+        int g = 0;  // first key tile of the unit, counted over all units
+        for (int u = blockIdx.x, i = 0; ok && u < p.units; u += gridDim.x, ++i, g += nk) {
+        int q0, h, b;
+        coords(u, q0, h, b);
         // logits of this thread's query row in log2 units: S * scale_log2, times the
         // row's RMSNorm factor when the queries arrive unnormalised
         float row_scale = p.scale_log2;
         if (p.qn.ssq) {
             const int qrow = q0 + 128 * t + r;
             if (qrow < p.Lq) {
-                const float* g = p.qn.ssq + ((long long)b * p.Lq + qrow) * p.qn.ssq_ld;
+                const float* gs = p.qn.ssq + ((long long)b * p.Lq + qrow) * p.qn.ssq_ld;
                 float ss = 0.f;
-                for (int k = 0; k < p.qn.ngroups; ++k) ss += __ldg(g + k);
+                for (int k = 0; k < p.qn.ngroups; ++k) ss += __ldg(gs + k);
                 row_scale *= rsqrtf(ss * p.qn.inv_n + p.qn.eps);
             }
         }
         float m_run = -INFINITY, l_run = 0.0f;
-        bool ok = true;
         for (int j = 0; j < nk; ++j) {
             // all tcgen05.ld/st below are warp-collective: the warp's decisions stay uniform
-            if (!__all_sync(0xffffffffu, mbar_wait(s_full + t, j & 1, abort_flag, p.wc))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full + t, (g + j) & 1, abort_flag, p.wc))) { ok = false; break; }
             tc_fence_after();
             uint32_t sv[4][32];
 #pragma unroll
@@ -341,7 +376,10 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full + t);
         }
-        if (ok && __all_sync(0xffffffffu, mbar_wait(o_final + t, 0, abort_flag, p.wc))) {
+        if (!ok) break;
+        // the unit's output: O_t / l once the last P.V of the unit has landed
+        if (!__all_sync(0xffffffffu, mbar_wait(o_final + t, i & 1, abort_flag, p.wc))) { ok = false; break; }
+        {
             tc_fence_after();
             const float inv = 1.0f / l_run;
             const int row = q0 + 128 * t + r;
@@ -354,14 +392,15 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                 if (row < p.Lq) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        dst[i] = make_uint4(pack_bf16(__uint_as_float(ov[8 * i]) * inv, __uint_as_float(ov[8 * i + 1]) * inv),
-                                            pack_bf16(__uint_as_float(ov[8 * i + 2]) * inv, __uint_as_float(ov[8 * i + 3]) * inv),
-                                            pack_bf16(__uint_as_float(ov[8 * i + 4]) * inv, __uint_as_float(ov[8 * i + 5]) * inv),
-                                            pack_bf16(__uint_as_float(ov[8 * i + 6]) * inv, __uint_as_float(ov[8 * i + 7]) * inv));
+                    for (int w = 0; w < 4; ++w) {
+                        dst[w] = make_uint4(pack_bf16(__uint_as_float(ov[8 * w]) * inv, __uint_as_float(ov[8 * w + 1]) * inv),
+                                            pack_bf16(__uint_as_float(ov[8 * w + 2]) * inv, __uint_as_float(ov[8 * w + 3]) * inv),
+                                            pack_bf16(__uint_as_float(ov[8 * w + 4]) * inv, __uint_as_float(ov[8 * w + 5]) * inv),
+                                            pack_bf16(__uint_as_float(ov[8 * w + 6]) * inv, __uint_as_float(ov[8 * w + 7]) * inv));
                     }
                 }
             }
+        }
         }
     }
 
@@ -371,7 +410,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
         // a wait gave up somewhere in the CTA: let this CTA's own loads and MMAs
         // land (bounded) before its shared and tensor memory are released
         if (warp == 0 && lane == 0) {
-            mbar_drain(q_full, 0, 200000000ull);
+            if (qpar >= 0) mbar_drain(q_full, static_cast<uint32_t>(qpar), 200000000ull);
             for (int s = 0; s < KSTAGES; ++s)
                 if (karmed & (1u << s)) mbar_drain(k_full + s, (kpar >> s) & 1, 200000000ull);
             for (int s = 0; s < VSTAGES; ++s)
@@ -418,13 +457,18 @@ cudaError_t launch_attention(const void* q, long long ldq, const void* k, long l
     p.Lq = Lq;
     p.Lk = Lk;
     p.heads = heads;
+    p.nqb = (Lq + 255) / 256;
+    p.units = p.nqb * heads * B;
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.ldo = ldo;
     p.scale_log2 = 1.4426950408889634f / sqrtf(128.0f);
     p.qn = qn;
     p.wc.err = ctx.err;
     p.wc.limit_ns = ctx.wait_limit_ns;
-    dim3 grid((Lq + 255) / 256, heads, B);
+    // one unit per CTA for long key sets; for up to 4 key tiles (the text
+    // tokens of the cross-attention) one CTA per SM walks the units
+    const int nk = (Lk + 127) / 128;
+    const int grid = nk <= 4 && p.units > ctx.num_sms ? ctx.num_sms : p.units;
     attn_tc_kernel<<<grid, attn::THREADS, attn::SMEM_BYTES, ctx.stream>>>(tq, tk, tv, p);
     if (ctx.launches) ++*ctx.launches;
     return cudaGetLastError();
