@@ -286,8 +286,16 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
 // ((x0, x1) -> (x0 cos - x1 sin, x1 cos + x0 sin)) when RoPE is on; the row
 // factor rsqrt(mean + eps) commutes with both and is applied later.  All of
 // it on packed fp32 pairs, so the scalar FP32 pipe stays free for MMA issue.
+// RoPE (cos, sin) of the 16 rotation pairs of a 32-column chunk at token
+// position (f, ii, jj), from the pair-major tables; loaded ahead of the chunk.
+__device__ __forceinline__ void qk_rope_load(const EpiParams& e, int c, int f, int ii, int jj, float2 (&cs)[16]) {
+    const int p0 = (c & 127) >> 1;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cs[i] = __ldg(rope_entry_pm(e.rope, p0 + i, f, ii, jj));
+}
+
 __device__ __forceinline__ float epilogue_qk_chunk(const EpiParams& e, int row, int c, const uint32_t (&r)[32],
-                                                   bool normed, int f, int ii, int jj) {
+                                                   bool normed, const float2 (&cs)[16]) {
     uint64_t v2[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) v2[i] = f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
@@ -315,11 +323,7 @@ __device__ __forceinline__ float epilogue_qk_chunk(const EpiParams& e, int row, 
             v2[2 * i] = mul2(v2[2 * i], g.x);
             v2[2 * i + 1] = mul2(v2[2 * i + 1], g.y);
         }
-        if (e.rope.t) {  // (pair-major tables) all 16 lookups in flight before any is used
-            const int p0 = (c & 127) >> 1;
-            float2 cs[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) cs[i] = __ldg(rope_entry_pm(e.rope, p0 + i, f, ii, jj));
+        if (e.rope.t) {  // cs loaded by the caller ahead of the accumulator chunk
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 float a, b;
@@ -419,13 +423,23 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, int row, int 
             jj = rem - ii * p.epi.rope.Wp;
         }
         float ss = 0.0f;
-#pragma unroll 1
-        for (int c0 = chalf * CW; c0 < (chalf + 1) * CW; c0 += 32) {
+        // the RoPE entries of chunk k + 1 load while chunk k is read out of tensor
+        // memory and computed (two buffers, each reused after its values are consumed)
+        const bool rope = normed && p.epi.rope.t;
+        float2 ca[16], cb[16];
+        auto chunk = [&](int k, float2 (&use)[16], float2 (&next)[16]) {
+            const int c0 = chalf * CW + k * 32;
             uint32_t r[32];
             tmem_ld32(taddr + c0, r);
+            if (k + 1 < CW / 32 && rope) qk_rope_load(p.epi, nb * BN + c0 + 32, f, ii, jj, next);
             tmem_ld_wait(r);
-            if (row < p.M) ss += epilogue_qk_chunk(p.epi, row, nb * BN + c0, r, normed, f, ii, jj);
-        }
+            if (row < p.M) ss += epilogue_qk_chunk(p.epi, row, nb * BN + c0, r, normed, use);
+        };
+        if (rope) qk_rope_load(p.epi, nb * BN + chalf * CW, f, ii, jj, ca);
+        chunk(0, ca, cb);
+        chunk(1, cb, ca);
+        chunk(2, ca, cb);
+        chunk(3, cb, ca);
         if (normed && row < p.M) p.epi.ssq[(long long)row * p.epi.ssq_ld + gcol / 128] = ss;
     } else {
 #pragma unroll 1
