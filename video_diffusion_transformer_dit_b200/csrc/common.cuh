@@ -110,7 +110,7 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint6
 
 // ----------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor) tile loads into this CTA's shared memory,
-// completing on an mbarrier.  No TMA load uses cluster multicast.
+// completing on an mbarrier; every load fills only this CTA's shared memory.
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -307,8 +307,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
 // SM pairs (clusters of two CTAs, tcgen05 .cta_group::2).  The two CTAs of a
 // pair have the same shared-memory layout; `mapa` turns the address of a
 // variable in this CTA into the address of the same variable in the other.
-// No TMA load here uses cluster multicast: each CTA loads its own half of
-// every operand tile into its own shared memory.
+// Each CTA loads its own half of every operand tile into its own shared
+// memory.
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
