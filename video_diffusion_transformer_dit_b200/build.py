@@ -2,11 +2,14 @@
 
 ``python -m video_diffusion_transformer_dit_b200.build`` compiles every
 ``csrc/*.cu`` into ``_build/`` and links ``libwandit.so`` next to this file.
-Objects are rebuilt when their source or any header changed.
+Objects are rebuilt when their source or any header changed.  Concurrent
+callers (one per rank under torchrun) serialise on a file lock in `_build/`:
+the first compiles, the others then find everything up to date.
 """
 from __future__ import annotations
 
 import concurrent.futures as cf
+import fcntl
 import glob
 import os
 import shutil
@@ -52,6 +55,15 @@ def _compile(src, obj, verbose):
 
 def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
+    with open(os.path.join(BUILD, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        try:
+            return _build_locked(force, verbose)
+        finally:
+            fcntl.flock(lock, fcntl.LOCK_UN)
+
+
+def _build_locked(force: bool, verbose: bool) -> str:
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdrs = _headers()
     jobs = []
