@@ -462,6 +462,27 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, int row, int 
 constexpr int EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
 
+// Residual epilogue with the residual read from the warp's shared-memory slab:
+// 32 rows (r = the thread's row in the slab) x 128 columns as two 64-column
+// boxes with the 128-byte swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)).
+template <int KIND>
+__device__ __forceinline__ void epilogue_tile_staged(const GemmParams& p, int row, int nb, uint32_t taddr, int chalf,
+                                                     const uint8_t* xs, int r) {
+    constexpr int BN = 256, CW = 128;
+#pragma unroll 1
+    for (int k = 0; k < CW / 32; ++k) {
+        const int c0 = chalf * CW + k * 32;
+        uint32_t acc[32];
+        tmem_ld32(taddr + c0, acc);
+        const uint8_t* rowp = xs + (k >> 1) * (32 * 128) + r * 128;
+        uint4 xu[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xu[i] = *reinterpret_cast<const uint4*>(rowp + (((4 * (k & 1) + i) ^ (r & 7)) << 4));
+        tmem_ld_wait(acc);
+        if (row < p.M) epilogue_chunk_f2<KIND>(p.epi, row, nb * BN + c0, acc, xu);
+    }
+}
+
 template <int BN, int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -661,30 +682,43 @@ namespace pair2 {
 constexpr int BN = 256;
 constexpr int HALF_BYTES = 128 * 64 * 2;      // one 128 x 64 bf16 operand tile
 constexpr int STAGE_BYTES = 2 * HALF_BYTES;   // A rows + W half
-constexpr int STAGES = 6;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int XSLAB_BYTES = 32 * 128 * 2;     // one epilogue warp's residual rows: 32 x 128 bf16
+// Residual epilogues stage each warp's residual slab in shared memory (two
+// 64-column TMA boxes, 128-byte swizzle), which leaves room for 5 ring stages.
+template <bool STAGE_X>
+struct Cfg {
+    static constexpr int STAGES = STAGE_X ? 5 : 6;
+    static constexpr int X_BYTES = STAGE_X ? EPI_WARPS * XSLAB_BYTES : 0;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + X_BYTES + 1024 + 256;
+};
 // loads a producer that issued n loads put into stage s
+template <int STAGES>
 __device__ __forceinline__ uint32_t loads_in_stage(uint32_t n, int s) {
     return n > (uint32_t)s ? (n - 1 - s) / STAGES + 1 : 0u;
 }
 }  // namespace pair2
 
+// tmX (residual epilogues): the residual / output matrix, 64 x 32 boxes.
 template <int KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmX, const GemmParams p) {
     using namespace pair2;
+    constexpr bool STAGE_X = reads_residual(KIND);
+    constexpr int STAGES = Cfg<STAGE_X>::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;                          // [STAGES] this CTA's 128 A rows x 64
     uint8_t* sB = smem + STAGES * HALF_BYTES;    // [STAGES] this CTA's 128 W rows x 64
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint8_t* sX = smem + STAGES * STAGE_BYTES;   // [EPI_WARPS] residual slabs (STAGE_X)
+    uint64_t* full = reinterpret_cast<uint64_t*>(sX + Cfg<STAGE_X>::X_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* xbar = drain + 1;                  // [EPI_WARPS] residual slab landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + EPI_WARPS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile uint32_t* loads_issued = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
 
@@ -703,11 +737,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             mbar_init(tempty + a, 2 * EPI_WARPS);
         }
         mbar_init(drain, 1);
+        for (int w = 0; w < EPI_WARPS; ++w) mbar_init(xbar + w, 1);
         *abort_flag = 0;
         *loads_issued = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (STAGE_X) tma_prefetch_desc(&tmX);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -752,7 +788,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             // the MMA commits that free this CTA's stages arrive here: wait for
             // the last of them so none lands after the CTA has exited
             for (int s = 0; ok && s < STAGES; ++s) {
-                const uint32_t c = loads_in_stage(n_loads, s);
+                const uint32_t c = loads_in_stage<STAGES>(n_loads, s);
                 if (c) ok = mbar_wait(empty + s, (c - 1) & 1u, abort_flag, p.wc);
             }
             *loads_issued = n_loads;
@@ -803,24 +839,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const int q = warp & 3;
         const int chalf = (warp - 2) >> 2;
         const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);
+        // residual epilogues: this warp's 32 rows x 128 columns of the residual,
+        // TMA-loaded into its slab ahead of the accumulator (the next tile's as
+        // soon as the current one has been read)
+        uint8_t* xs = sX + (warp - 2) * XSLAB_BYTES;
+        uint64_t* xb = xbar + (warp - 2);
+        uint32_t xpar = 0;
+        bool xarmed = false;
+        auto load_x = [&](int tile) {
+            int mb, nb;
+            tile_coords(tile, p, mb, nb);
+            if (lane == 0) {
+                const int r0 = mb * 256 + static_cast<int>(rank) * 128 + q * 32, c0 = nb * BN + chalf * 128;
+                fence_proxy_async_smem();  // the slab's previous contents were read through the generic proxy
+                mbar_expect_tx(xb, XSLAB_BYTES);
+                tma_load_2d(xs, &tmX, xb, c0, r0);
+                tma_load_2d(xs + XSLAB_BYTES / 2, &tmX, xb, c0 + 64, r0);
+            }
+            xarmed = true;
+        };
+        if (STAGE_X && cid < p.num_tiles) load_x(cid);
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = cid; tile < p.num_tiles; tile += ncl) {
             int mb, nb;
             tile_coords(tile, p, mb, nb);
             const int row = mb * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
-            uint4 x0[4];
-            epilogue_prefetch<BN, KIND>(p, row, nb, chalf, x0);
             if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc))) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-            epilogue_tile<BN, KIND, false>(p, row, nb, taddr, chalf, x0);
+            if constexpr (STAGE_X) {
+                if (!__all_sync(0xffffffffu, mbar_wait(xb, xpar, abort_flag, p.wc))) break;
+                xarmed = false;
+                xpar ^= 1;
+                epilogue_tile_staged<KIND>(p, row, nb, taddr, chalf, xs, lane);
+            } else {
+                uint4 x0[4];
+                epilogue_tile<BN, KIND, false>(p, row, nb, taddr, chalf, x0);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(tempty0 + 8u * acc);
+            if (STAGE_X && tile + ncl < p.num_tiles) load_x(tile + ncl);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
+        // a slab load still in flight lands before the CTA's shared memory is released
+        if (xarmed && lane == 0) mbar_drain(xb, xpar, 200000000ull);
     }
 
     __syncthreads();
@@ -838,7 +903,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             const uint32_t n0 = *loads_issued;
             const uint32_t n1 = ld_shared_cluster_u32(mapa_shared(smem_u32((const void*)loads_issued), 1));
             for (int s = 0; s < STAGES; ++s) {
-                const uint32_t c0 = loads_in_stage(n0, s), c1 = loads_in_stage(n1, s);
+                const uint32_t c0 = loads_in_stage<STAGES>(n0, s), c1 = loads_in_stage<STAGES>(n1, s);
                 const uint32_t c = c0 > c1 ? c0 : c1;
                 if (!c) continue;
                 if (c0 > c1) mbar_complete_tx(full + s, STAGE_BYTES);
@@ -884,7 +949,7 @@ static int g_pair_clusters = 0;
 template <int KIND>
 static cudaError_t set_pair_attr_one() {
     return cudaFuncSetAttribute(gemm_pair_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                pair2::SMEM_BYTES);
+                                pair2::Cfg<reads_residual(KIND)>::SMEM_BYTES);
 }
 
 static cudaError_t init_pair_gemm() {
@@ -900,7 +965,7 @@ static cudaError_t init_pair_gemm() {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = pair2::SMEM_BYTES;
+    cfg.dynamicSmemBytes = pair2::Cfg<false>::SMEM_BYTES;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_tc_kernel<EPI_BIAS>, &cfg) != cudaSuccess) {
         cudaGetLastError();
@@ -1001,10 +1066,16 @@ cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long l
     if (!make_tmap_2d(&tb, W, K, N, ldw, 64, use_pair ? 128 : BN)) return cudaErrorInvalidValue;
     if (use_pair) {
         const int clusters = p.num_tiles < g_pair_clusters ? p.num_tiles : g_pair_clusters;
+        // residual epilogues read the residual tile through TMA (32-row x 64-column boxes)
+        CUtensorMap tx = ta;
+        if (reads_residual(epi.kind) &&
+            !make_tmap_2d(&tx, epi.out, (uint64_t)N, (uint64_t)M, (uint64_t)epi.ldo, 64, 32))
+            return cudaErrorInvalidValue;
         switch (epi.kind) {
-#define WAN_PAIR_CASE(K)                                                                                 \
-    case K:                                                                                              \
-        gemm_pair_tc_kernel<K><<<2 * clusters, GEMM_THREADS, pair2::SMEM_BYTES, ctx.stream>>>(ta, tb, p); \
+#define WAN_PAIR_CASE(K)                                                                                   \
+    case K:                                                                                                \
+        gemm_pair_tc_kernel<K><<<2 * clusters, GEMM_THREADS, pair2::Cfg<reads_residual(K)>::SMEM_BYTES,     \
+                                 ctx.stream>>>(ta, tb, tx, p);                                             \
         break;
             WAN_PAIR_CASE(EPI_BIAS)
             WAN_PAIR_CASE(EPI_BIAS_GELU)
