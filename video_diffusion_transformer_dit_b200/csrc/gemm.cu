@@ -59,6 +59,24 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmParams& p, int& 
 // pairs; bias, GELU, gate and residual run as f32x2 operations, which keeps
 // the scalar FP32 pipe free for the MMA-issuing warp on the same SM
 // sub-partitions (scalar FFMA traffic there slows tcgen05.mma issue).
+// Where the four 16-byte words (8 bf16 each) of an epilogue chunk go: the
+// row in global memory, or the row of an epilogue warp's shared-memory slab
+// (128-byte swizzle: 16-byte chunk j of slab row r at chunk j ^ (r & 7)).
+struct GlobalOut {
+    uint4* p;
+    __device__ __forceinline__ void put(int i, const uint4& w) const { p[i] = w; }
+};
+struct SlabOut {
+    uint8_t* rowp;  // slab row (box base + r * 128)
+    int j0, r7;     // first 16-byte chunk of the 32 columns, r & 7
+    __device__ __forceinline__ void put(int i, const uint4& w) const {
+        *reinterpret_cast<uint4*>(rowp + (((j0 + i) ^ r7) << 4)) = w;
+    }
+};
+__device__ __forceinline__ GlobalOut global_out(const EpiParams& e, int row, int c) {
+    return GlobalOut{reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c)};
+}
+
 // Residual rows of one 32-column chunk (4 x 16 B), loaded ahead of their use.
 __device__ __forceinline__ void load_residual(const EpiParams& e, int row, int c, uint4 (&xu)[4]) {
     const uint4* xp = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
@@ -66,9 +84,9 @@ __device__ __forceinline__ void load_residual(const EpiParams& e, int row, int c
     for (int i = 0; i < 4; ++i) xu[i] = xp[i];
 }
 
-template <int KIND>
+template <int KIND, class Out>
 __device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, int c, const uint32_t (&r)[32],
-                                                  const uint4 (&xu)[4]) {
+                                                  const uint4 (&xu)[4], const Out& out) {
     uint64_t v2[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) v2[i] = f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
@@ -86,7 +104,6 @@ __device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, i
 #pragma unroll
             for (int i = 0; i < 16; ++i) v2[i] = gelu_tanh_f2(v2[i]);
         }
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             uint32_t w[4];
@@ -96,10 +113,9 @@ __device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, i
                 f2unpack(v2[4 * i + h], a, b);
                 w[h] = pack_bf16(a, b);
             }
-            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            out.put(i, make_uint4(w[0], w[1], w[2], w[3]));
         }
     } else {  // EPI_GATE_RESIDUAL, EPI_RESIDUAL: x (4 x 16 B) arrives preloaded
-        uint4* xp = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
         const ulonglong2* g1 =
             e.gate1 ? reinterpret_cast<const ulonglong2*>(e.gate1 + (long long)(row / e.mod_div) * e.mod_ld + c) : nullptr;
         const ulonglong2* g0 = e.gate0 ? reinterpret_cast<const ulonglong2*>(e.gate0 + c) : nullptr;
@@ -141,7 +157,7 @@ __device__ __forceinline__ void epilogue_chunk_f2(const EpiParams& e, int row, i
                 f2unpack(o2, a, b);
                 ow[h] = pack_bf16(a, b);
             }
-            xp[i] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            out.put(i, make_uint4(ow[0], ow[1], ow[2], ow[3]));
         }
     }
 }
@@ -151,7 +167,7 @@ template <int KIND>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int c, const uint32_t (&r)[32]) {
     if constexpr (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU) {
         const uint4 none[4] = {};
-        epilogue_chunk_f2<KIND>(e, row, c, r, none);
+        epilogue_chunk_f2<KIND>(e, row, c, r, none, global_out(e, row, c));
     } else {
     float v[32];
 #pragma unroll
@@ -286,6 +302,16 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& e, int row, int 
 // ((x0, x1) -> (x0 cos - x1 sin, x1 cos + x0 sin)) when RoPE is on; the row
 // factor rsqrt(mean + eps) commutes with both and is applied later.  All of
 // it on packed fp32 pairs, so the scalar FP32 pipe stays free for MMA issue.
+// (frame, row, column) of the token of GEMM row `row` in the RoPE grid.
+__device__ __forceinline__ void qk_position(const EpiParams& e, int row, int& f, int& ii, int& jj) {
+    const int hw = e.rope.Hp * e.rope.Wp;
+    const int l = min(e.rope_tok0 + row % e.rope_L, e.rope.Fp * hw - 1);
+    f = l / hw;
+    const int rem = l - f * hw;
+    ii = rem / e.rope.Wp;
+    jj = rem - ii * e.rope.Wp;
+}
+
 // RoPE (cos, sin) of the 16 rotation pairs of a 32-column chunk at token
 // position (f, ii, jj), from the pair-major tables; loaded ahead of the chunk.
 __device__ __forceinline__ void qk_rope_load(const EpiParams& e, int c, int f, int ii, int jj, float2 (&cs)[16]) {
@@ -294,8 +320,9 @@ __device__ __forceinline__ void qk_rope_load(const EpiParams& e, int c, int f, i
     for (int i = 0; i < 16; ++i) cs[i] = __ldg(rope_entry_pm(e.rope, p0 + i, f, ii, jj));
 }
 
-__device__ __forceinline__ float epilogue_qk_chunk(const EpiParams& e, int row, int c, const uint32_t (&r)[32],
-                                                   bool normed, const float2 (&cs)[16]) {
+template <class Out>
+__device__ __forceinline__ float epilogue_qk_chunk(const EpiParams& e, int c, const uint32_t (&r)[32], bool normed,
+                                                   const float2 (&cs)[16], const Out& out) {
     uint64_t v2[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) v2[i] = f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
@@ -332,7 +359,6 @@ __device__ __forceinline__ float epilogue_qk_chunk(const EpiParams& e, int row, 
             }
         }
     }
-    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.out) + (long long)row * e.ldo + c);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         uint32_t w[4];
@@ -342,7 +368,7 @@ __device__ __forceinline__ float epilogue_qk_chunk(const EpiParams& e, int row, 
             f2unpack(v2[4 * i + h], a, b);
             w[h] = pack_bf16(a, b);
         }
-        dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        out.put(i, make_uint4(w[0], w[1], w[2], w[3]));
     }
     return ss;
 }
@@ -375,6 +401,11 @@ __device__ __forceinline__ void epilogue_cfg_euler(const EpiParams& e, int row, 
 }
 
 __host__ __device__ constexpr bool reads_residual(int kind) { return kind == EPI_GATE_RESIDUAL || kind == EPI_RESIDUAL; }
+// SM-pair epilogues that go through a shared-memory slab per warp (TMA-loaded
+// residual, TMA-stored results; 5 ring stages): the residual and q/k-norm
+// kinds.  Bias and GELU keep 6 stages and store from registers (their long-K
+// or wide-N mainloops gained nothing from the slab and lost a ring stage).
+__host__ __device__ constexpr bool uses_slab(int kind) { return reads_residual(kind) || kind == EPI_QK_NORM; }
 
 // Residual of the first chunk of an epilogue warp's share of tile (row, nb),
 // loaded before the warp waits for the accumulator.
@@ -402,7 +433,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, int row, int 
             uint32_t r[32];
             tmem_ld32(taddr + c0, r);
             tmem_ld_wait(r);
-            if (row < p.M) epilogue_chunk_f2<KIND>(p.epi, row, nb * BN + c0, r, use);
+            if (row < p.M) epilogue_chunk_f2<KIND>(p.epi, row, nb * BN + c0, r, use, global_out(p.epi, row, nb * BN + c0));
         };
         chunk(0, x0, x1);
         if constexpr (CW / 32 > 1) chunk(1, x1, x0);
@@ -414,14 +445,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, int row, int 
         const int gcol = nb * BN + chalf * CW;
         const bool normed = gcol < p.epi.norm_cols;
         int f = 0, ii = 0, jj = 0;
-        if (normed && p.epi.rope.t) {
-            const int hw = p.epi.rope.Hp * p.epi.rope.Wp;
-            const int l = min(p.epi.rope_tok0 + row % p.epi.rope_L, p.epi.rope.Fp * hw - 1);
-            f = l / hw;
-            const int rem = l - f * hw;
-            ii = rem / p.epi.rope.Wp;
-            jj = rem - ii * p.epi.rope.Wp;
-        }
+        if (normed && p.epi.rope.t) qk_position(p.epi, row, f, ii, jj);
         float ss = 0.0f;
         // the RoPE entries of chunk k + 1 load while chunk k is read out of tensor
         // memory and computed (two buffers, each reused after its values are consumed)
@@ -433,7 +457,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, int row, int 
             tmem_ld32(taddr + c0, r);
             if (k + 1 < CW / 32 && rope) qk_rope_load(p.epi, nb * BN + c0 + 32, f, ii, jj, next);
             tmem_ld_wait(r);
-            if (row < p.M) ss += epilogue_qk_chunk(p.epi, row, nb * BN + c0, r, normed, use);
+            if (row < p.M) ss += epilogue_qk_chunk(p.epi, nb * BN + c0, r, normed, use, global_out(p.epi, row, nb * BN + c0));
         };
         if (rope) qk_rope_load(p.epi, nb * BN + chalf * CW, f, ii, jj, ca);
         chunk(0, ca, cb);
@@ -462,24 +486,51 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, int row, int 
 constexpr int EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
 
-// Residual epilogue with the residual read from the warp's shared-memory slab:
-// 32 rows (r = the thread's row in the slab) x 128 columns as two 64-column
-// boxes with the 128-byte swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)).
+// SM-pair epilogue of one warp's share of a tile through its shared-memory
+// slab: 32 rows (r = the thread's row in the slab) x 128 columns as two
+// 64-column boxes with the 128-byte swizzle.  Residual kinds read x from the
+// slab (TMA-loaded by the caller); every kind writes its bf16 results into the
+// slab, which the caller then stores with TMA.
 template <int KIND>
-__device__ __forceinline__ void epilogue_tile_staged(const GemmParams& p, int row, int nb, uint32_t taddr, int chalf,
-                                                     const uint8_t* xs, int r) {
+__device__ __forceinline__ void epilogue_tile_slab(const GemmParams& p, int row, int nb, uint32_t taddr, int chalf,
+                                                   uint8_t* xs, int r) {
     constexpr int BN = 256, CW = 128;
+    const int r7 = r & 7;
+    auto slab = [&](int k) { return SlabOut{xs + (k >> 1) * (32 * 128) + r * 128, 4 * (k & 1), r7}; };
+    if constexpr (KIND == EPI_QK_NORM) {
+        const int gcol = nb * BN + chalf * CW;
+        const bool normed = gcol < p.epi.norm_cols;
+        int f = 0, ii = 0, jj = 0;
+        if (normed && p.epi.rope.t) qk_position(p.epi, row, f, ii, jj);
+        float ss = 0.0f;
+        const bool rope = normed && p.epi.rope.t;
 #pragma unroll 1
-    for (int k = 0; k < CW / 32; ++k) {
-        const int c0 = chalf * CW + k * 32;
-        uint32_t acc[32];
-        tmem_ld32(taddr + c0, acc);
-        const uint8_t* rowp = xs + (k >> 1) * (32 * 128) + r * 128;
-        uint4 xu[4];
+        for (int k = 0; k < CW / 32; ++k) {
+            // the chunk's 16 RoPE entries load while its accumulator columns are read out
+            const int c0 = chalf * CW + k * 32;
+            uint32_t acc[32];
+            float2 cs[16];
+            tmem_ld32(taddr + c0, acc);
+            if (rope) qk_rope_load(p.epi, nb * BN + c0, f, ii, jj, cs);
+            tmem_ld_wait(acc);
+            if (row < p.M) ss += epilogue_qk_chunk(p.epi, nb * BN + c0, acc, normed, cs, slab(k));
+        }
+        if (normed && row < p.M) p.epi.ssq[(long long)row * p.epi.ssq_ld + gcol / 128] = ss;
+    } else {
+#pragma unroll 1
+        for (int k = 0; k < CW / 32; ++k) {
+            const int c0 = chalf * CW + k * 32;
+            uint32_t acc[32];
+            tmem_ld32(taddr + c0, acc);
+            uint4 xu[4] = {};
+            if constexpr (reads_residual(KIND)) {
+                const SlabOut s = slab(k);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) xu[i] = *reinterpret_cast<const uint4*>(rowp + (((4 * (k & 1) + i) ^ (r & 7)) << 4));
-        tmem_ld_wait(acc);
-        if (row < p.M) epilogue_chunk_f2<KIND>(p.epi, row, nb * BN + c0, acc, xu);
+                for (int i = 0; i < 4; ++i) xu[i] = *reinterpret_cast<const uint4*>(s.rowp + (((s.j0 + i) ^ r7) << 4));
+            }
+            tmem_ld_wait(acc);
+            if (row < p.M) epilogue_chunk_f2<KIND>(p.epi, row, nb * BN + c0, acc, xu, slab(k));
+        }
     }
 }
 
@@ -705,7 +756,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmX, const GemmParams p) {
     using namespace pair2;
-    constexpr bool STAGE_X = reads_residual(KIND);
+    constexpr bool STAGE_X = uses_slab(KIND);
     constexpr int STAGES = Cfg<STAGE_X>::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -839,18 +890,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const int q = warp & 3;
         const int chalf = (warp - 2) >> 2;
         const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);
-        // residual epilogues: this warp's 32 rows x 128 columns of the residual,
-        // TMA-loaded into its slab ahead of the accumulator (the next tile's as
-        // soon as the current one has been read)
+        // each epilogue warp owns a slab of 32 rows x 128 columns: residual kinds
+        // TMA-load the tile's x into it ahead of the accumulator (the next tile's as
+        // soon as the current one has been stored), every kind writes its results
+        // into it and stores them with TMA
         uint8_t* xs = sX + (warp - 2) * XSLAB_BYTES;
         uint64_t* xb = xbar + (warp - 2);
         uint32_t xpar = 0;
-        bool xarmed = false;
-        auto load_x = [&](int tile) {
+        bool xarmed = false, stored = false;
+        auto slab_coords = [&](int tile, int& c0, int& r0) {
             int mb, nb;
             tile_coords(tile, p, mb, nb);
+            r0 = mb * 256 + static_cast<int>(rank) * 128 + q * 32;
+            c0 = nb * BN + chalf * 128;
+        };
+        auto load_x = [&](int tile) {
+            int c0, r0;
+            slab_coords(tile, c0, r0);
             if (lane == 0) {
-                const int r0 = mb * 256 + static_cast<int>(rank) * 128 + q * 32, c0 = nb * BN + chalf * 128;
                 fence_proxy_async_smem();  // the slab's previous contents were read through the generic proxy
                 mbar_expect_tx(xb, XSLAB_BYTES);
                 tma_load_2d(xs, &tmX, xb, c0, r0);
@@ -858,7 +915,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             }
             xarmed = true;
         };
-        if (STAGE_X && cid < p.num_tiles) load_x(cid);
+        // the previous tile's store has read the slab (before it is rewritten)
+        auto slab_free = [&]() {
+            if (stored && lane == 0) bulk_wait_read_all();
+            __syncwarp();
+        };
+        if (STAGE_X && reads_residual(KIND) && cid < p.num_tiles) load_x(cid);
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = cid; tile < p.num_tiles; tile += ncl) {
@@ -868,23 +930,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.wc))) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-            if constexpr (STAGE_X) {
-                if (!__all_sync(0xffffffffu, mbar_wait(xb, xpar, abort_flag, p.wc))) break;
-                xarmed = false;
-                xpar ^= 1;
-                epilogue_tile_staged<KIND>(p, row, nb, taddr, chalf, xs, lane);
-            } else {
+            if constexpr (!STAGE_X) {  // bias / GELU: results stored from registers
                 uint4 x0[4];
                 epilogue_tile<BN, KIND, false>(p, row, nb, taddr, chalf, x0);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(tempty0 + 8u * acc);
+            } else {
+                if constexpr (reads_residual(KIND)) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(xb, xpar, abort_flag, p.wc))) break;
+                    xarmed = false;
+                    xpar ^= 1;
+                } else {
+                    slab_free();
+                }
+                epilogue_tile_slab<KIND>(p, row, nb, taddr, chalf, xs, lane);
+                tc_fence_before();
+                fence_proxy_async_smem();  // the slab's results, written through the generic proxy, go out by TMA
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_remote(tempty0 + 8u * acc);
+                    int c0, r0;
+                    slab_coords(tile, c0, r0);
+                    tma_store_2d(&tmX, xs, c0, r0);
+                    tma_store_2d(&tmX, xs + XSLAB_BYTES / 2, c0 + 64, r0);
+                    bulk_commit();
+                }
+                stored = true;
+                if (reads_residual(KIND) && tile + ncl < p.num_tiles) {
+                    slab_free();
+                    load_x(tile + ncl);
+                }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(tempty0 + 8u * acc);
-            if (STAGE_X && tile + ncl < p.num_tiles) load_x(tile + ncl);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
-        // a slab load still in flight lands before the CTA's shared memory is released
+        // stores complete and a slab load still in flight lands before the CTA's
+        // shared memory is released
+        if (stored && lane == 0) bulk_wait_all();
         if (xarmed && lane == 0) mbar_drain(xb, xpar, 200000000ull);
     }
 
@@ -949,7 +1032,7 @@ static int g_pair_clusters = 0;
 template <int KIND>
 static cudaError_t set_pair_attr_one() {
     return cudaFuncSetAttribute(gemm_pair_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                pair2::Cfg<reads_residual(KIND)>::SMEM_BYTES);
+                                pair2::Cfg<uses_slab(KIND)>::SMEM_BYTES);
 }
 
 static cudaError_t init_pair_gemm() {
@@ -1043,9 +1126,15 @@ cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long l
             (epi.rope.t && epi.rope_L <= 0))
             return cudaErrorInvalidValue;
     }
-    const bool use_pair = ctx.gemm_pair && g_pair_clusters > 0 && BN == 256 && M >= 512 &&
-                          (epi.kind == EPI_BIAS || epi.kind == EPI_BIAS_GELU || epi.kind == EPI_GATE_RESIDUAL ||
-                           epi.kind == EPI_RESIDUAL || epi.kind == EPI_QK_NORM);
+    bool use_pair = ctx.gemm_pair && g_pair_clusters > 0 && BN == 256 && M >= 512 &&
+                    (epi.kind == EPI_BIAS || epi.kind == EPI_BIAS_GELU || epi.kind == EPI_GATE_RESIDUAL ||
+                     epi.kind == EPI_RESIDUAL || epi.kind == EPI_QK_NORM);
+    // the pair epilogue loads residuals and stores results through TMA (32-row x
+    // 64-column boxes of the bf16 output); an output TMA cannot describe (a
+    // pointer or row stride off 16 bytes) takes the single-SM tiles instead
+    CUtensorMap tx;
+    if (use_pair && !make_tmap_2d(&tx, epi.out, (uint64_t)N, (uint64_t)M, (uint64_t)epi.ldo, 64, 32))
+        use_pair = false;
     GemmParams p;
     p.M = M;
     p.N = N;
@@ -1066,15 +1155,10 @@ cudaError_t launch_gemm(const void* A, long long lda, const void* W, long long l
     if (!make_tmap_2d(&tb, W, K, N, ldw, 64, use_pair ? 128 : BN)) return cudaErrorInvalidValue;
     if (use_pair) {
         const int clusters = p.num_tiles < g_pair_clusters ? p.num_tiles : g_pair_clusters;
-        // residual epilogues read the residual tile through TMA (32-row x 64-column boxes)
-        CUtensorMap tx = ta;
-        if (reads_residual(epi.kind) &&
-            !make_tmap_2d(&tx, epi.out, (uint64_t)N, (uint64_t)M, (uint64_t)epi.ldo, 64, 32))
-            return cudaErrorInvalidValue;
         switch (epi.kind) {
 #define WAN_PAIR_CASE(K)                                                                                   \
     case K:                                                                                                \
-        gemm_pair_tc_kernel<K><<<2 * clusters, GEMM_THREADS, pair2::Cfg<reads_residual(K)>::SMEM_BYTES,     \
+        gemm_pair_tc_kernel<K><<<2 * clusters, GEMM_THREADS, pair2::Cfg<uses_slab(K)>::SMEM_BYTES,         \
                                  ctx.stream>>>(ta, tb, tx, p);                                             \
         break;
             WAN_PAIR_CASE(EPI_BIAS)
