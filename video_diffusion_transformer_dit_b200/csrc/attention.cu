@@ -60,8 +60,10 @@ constexpr int SBAR = SV + VSTAGES * TILE_BYTES;
 constexpr int SMEM_BYTES = SBAR + 256 + 1024;
 constexpr int THREADS = 384;
 constexpr int REGS_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
-constexpr int REGS_CONTROL = 96;   // warpgroup 0: producer + MMA issuer
-constexpr int REGS_SOFTMAX = 200;  // warpgroups 1, 2
+// warpgroup 0 (producer + MMA issuer) / warpgroups 1, 2 (softmax); 88 for the
+// first spilled in the issuer and measured 1-2 % slower than 96 / 200
+constexpr int REGS_CONTROL = 96;
+constexpr int REGS_SOFTMAX = 200;
 static_assert(128 * REGS_CONTROL + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH, "register split");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 // P.V of a key tile goes in two K = 64 halves, the first issued as soon as the
@@ -178,6 +180,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                 varmed |= 1u << vs;
                 vpar = (vpar & ~(1u << vs)) | (vp << vs);
             }
+                if constexpr (!SPLIT_S) break;  // one unit per CTA
             }
         }
     } else if (warp == 1) {
@@ -286,6 +289,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                     }
                 }
             }
+            if constexpr (!SPLIT_S) break;  // one unit per CTA
         }
     }
     } else {
@@ -432,6 +436,7 @@ __global__ void __launch_bounds__(attn::THREADS, 1)
                 }
             }
         }
+            if constexpr (!SPLIT_S) break;  // one unit per CTA
         }
     }
 
