@@ -12,7 +12,7 @@
 // (the next unit's Q loads as soon as the last S MMA of the current one has
 // read Q), K / V / S / P once per key tile.  12 warps in
 // three warpgroups; the first gives registers to the two softmax groups
-// (96 / 200 / 200 per thread, 63488 of the 384 x 168 = 64512 at launch):
+// (104 / 192 / 192 per thread, 62464 of the 384 x 168 = 64512 at launch):
 //   warp 0      TMA producer: both Q tiles of a unit, then K and V tiles of 128
 //               keys in two-slot rings (3-D tensor maps: rows past the
 //               sequence read as zero);
@@ -60,10 +60,12 @@ constexpr int SBAR = SV + VSTAGES * TILE_BYTES;
 constexpr int SMEM_BYTES = SBAR + 256 + 1024;
 constexpr int THREADS = 384;
 constexpr int REGS_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
-// warpgroup 0 (producer + MMA issuer) / warpgroups 1, 2 (softmax); 88 for the
-// first spilled in the issuer and measured 1-2 % slower than 96 / 200
-constexpr int REGS_CONTROL = 96;
-constexpr int REGS_SOFTMAX = 200;
+// warpgroup 0 (producer + MMA issuer) / warpgroups 1, 2 (softmax), measured in
+// the 480p step: 88 / 208 spilled in the issuer (1-2 % slower than 96 / 200),
+// 104 / 192 ran 0.8 % faster than 96 / 200 and level with 120 / 192, 112 / 184
+// spills in the softmax
+constexpr int REGS_CONTROL = 104;
+constexpr int REGS_SOFTMAX = 192;
 static_assert(128 * REGS_CONTROL + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH, "register split");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 // P.V of a key tile goes in two K = 64 halves, the first issued as soon as the
