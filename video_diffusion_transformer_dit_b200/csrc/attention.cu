@@ -476,6 +476,7 @@ cudaError_t init_kernel_attributes() {
         e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn::SMEM_BYTES);
     if (e == cudaSuccess) e = init_gemm_attributes();
     if (e == cudaSuccess) e = init_conv_attributes();
+    if (e == cudaSuccess) e = init_layernorm_attributes();
     return e;
 }
 

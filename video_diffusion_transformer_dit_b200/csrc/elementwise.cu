@@ -100,22 +100,36 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __r
     }
 }
 
-// LayerNorm modes 1 and 2 for D <= 1536, each warp walking `rpw` consecutive rows
-// (a grid of one 256-thread CTA per SM).  The warp's columns of the
-// modulation (or affine) vectors stay in registers and are reloaded only when
-// the rows cross into the next sample, so per row only x and y move through
-// L1 (the per-row reload of 8 bytes of fp32 vectors per element made the
-// one-row-per-warp kernel L1-bound); rows are loaded two ahead of their use.
+// LayerNorm modes 1 and 2 for D <= 1536, each warp walking `rpw` consecutive
+// rows (a grid of one 256-thread CTA per SM).  The warp's columns of the
+// modulation (or affine) vectors stay in registers and are reloaded only where
+// the rows cross into the next sample, so per row only x and y move through L1
+// (the per-row reload of 8 bytes of fp32 vectors per element made the
+// one-row-per-warp kernel L1-bound).  Rows arrive through a ring of LN_RING
+// shared-memory row buffers per warp, each filled by one bulk copy issued
+// LN_RING rows ahead (bounded waits; no registers held for rows in flight).
+constexpr int LN_RING = 4;
+constexpr int LN_ROW_BYTES = 1536 * 2;
+constexpr int LN_SMEM = 8 * LN_RING * LN_ROW_BYTES + 8 * LN_RING * 8 + 16;
 template <int NCH, int MODE>
 __global__ void __launch_bounds__(256, 1)
     layernorm_rows_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y, int rows, int rpw,
-                          float eps, const float* gamma, const float* beta, const float* shift0, const float* shift1,
-                          const float* scale0, const float* scale1, int mod_div, long long mod_ld) {
+                          float eps, const float* gamma, const float* beta, const float* shift1,
+                          const float* scale1, int mod_div, long long mod_ld, WaitCtl wc) {
     constexpr int D = NCH * 256;
+    extern __shared__ __align__(128) uint8_t ln_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t* ring = ln_smem + warp * LN_RING * LN_ROW_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(ln_smem + 8 * LN_RING * LN_ROW_BYTES) + warp * LN_RING;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(ln_smem + 8 * LN_RING * LN_ROW_BYTES + 8 * LN_RING * 8);
+    if (threadIdx.x == 0) *abort_flag = 0;
+    if (lane == 0) {
+        for (int k = 0; k < LN_RING; ++k) mbar_init(bars + k, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
     const int r0 = (blockIdx.x * 8 + warp) * rpw;
     const int r1 = min(r0 + rpw, rows);
-    if (r0 >= r1) return;
     float ga[NCH][8], gb[NCH][8];  // y = (x - mean) * rstd * ga + gb on this lane's columns
     long long m_cur = -1;
     auto load_mod = [&](long long m) {
@@ -131,15 +145,30 @@ __global__ void __launch_bounds__(256, 1)
             }
         }
     };
-    auto load_row = [&](int row, uint4 (&u)[NCH]) {
-        if (row < r1) {
-            const __nv_bfloat16* xr = x + (long long)row * D;
-#pragma unroll
-            for (int t = 0; t < NCH; ++t) u[t] = *reinterpret_cast<const uint4*>(xr + (t * 32 + lane) * 8);
-        }
+    auto fetch = [&](int row) {  // lane 0: the row into its ring slot
+        const int k = (row - r0) % LN_RING;
+        mbar_expect_tx(bars + k, D * 2);
+        bulk_load(ring + k * LN_ROW_BYTES, x + (long long)row * D, D * 2, bars + k);
     };
-    auto do_row = [&](int row, const uint4 (&u)[NCH]) {
-        if (row >= r1) return;
+    if (MODE == 1) load_mod(0);
+    int issued = r0;  // rows whose copy has been issued: [r0, issued)
+    if (lane == 0)
+        for (; issued < r1 && issued < r0 + LN_RING; ++issued) fetch(issued);
+    issued = __shfl_sync(0xffffffffu, issued, 0);
+    int row = r0;
+    for (; row < r1; ++row) {
+        const int n = row - r0, k = n % LN_RING;
+        if (!__all_sync(0xffffffffu, mbar_wait(bars + k, (n / LN_RING) & 1, abort_flag, wc))) break;
+        uint4 u[NCH];
+        const uint8_t* src = ring + k * LN_ROW_BYTES;
+#pragma unroll
+        for (int t = 0; t < NCH; ++t) u[t] = *reinterpret_cast<const uint4*>(src + (t * 32 + lane) * 16);
+        __syncwarp();  // the slot is read: refill it with the row LN_RING ahead
+        if (lane == 0 && issued < r1) {
+            fence_proxy_async_smem();
+            fetch(issued);
+        }
+        ++issued;
         if (MODE != 1) {
             const long long m = (long long)(row / mod_div) * mod_ld;
             if (m != m_cur) {
@@ -177,19 +206,32 @@ __global__ void __launch_bounds__(256, 1)
             for (int i = 0; i < 8; ++i) o[i] = (v[i] - mean) * rstd * ga[t][i] + gb[t][i];
             store8(yr + (t * 32 + lane) * 8, o);
         }
-    };
-    if (MODE == 1) load_mod(0);
-    uint4 ua[NCH], ub[NCH], uc[NCH];
-    load_row(r0, ua);
-    load_row(r0 + 1, ub);
-    for (int row = r0; row < r1; row += 3) {  // three buffers: each is refilled right after its row is done
-        load_row(row + 2, uc);
-        do_row(row, ua);
-        load_row(row + 3, ua);
-        do_row(row + 1, ub);
-        load_row(row + 4, ub);
-        do_row(row + 2, uc);
     }
+    // after a wait gave up, the copies in flight (rows from the one not waited for
+    // up to the last issued, one per ring slot) land before the CTA exits
+    if (row < r1 && lane == 0) {
+        for (int rr = row; rr < min(issued, r1); ++rr) {
+            const int n = rr - r0;
+            mbar_drain(bars + n % LN_RING, (n / LN_RING) & 1, 200000000ull);
+        }
+    }
+}
+
+template <int NCH>
+static cudaError_t set_ln_rows_attr() {
+    cudaError_t e = cudaFuncSetAttribute(layernorm_rows_kernel<NCH, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, LN_SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(layernorm_rows_kernel<NCH, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, LN_SMEM);
+    return e;
+}
+
+cudaError_t init_layernorm_attributes() {
+    cudaError_t e = set_ln_rows_attr<1>();
+    if (e == cudaSuccess) e = set_ln_rows_attr<2>();
+    if (e == cudaSuccess) e = set_ln_rows_attr<3>();
+    if (e == cudaSuccess) e = set_ln_rows_attr<4>();
+    if (e == cudaSuccess) e = set_ln_rows_attr<6>();
+    return e;
 }
 
 cudaError_t launch_layernorm(const void* x, void* y, int rows, int D, float eps, int mode, const float* gamma,
@@ -207,14 +249,15 @@ cudaError_t launch_layernorm(const void* x, void* y, int rows, int D, float eps,
         const int warps = 8 * ctx.num_sms;
         const int rpw = (rows + warps - 1) / warps;
         const int blocks = (rows + 8 * rpw - 1) / (8 * rpw);
-#define WAN_LN_ROWS(n)                                                                                          \
-    case n:                                                                                                     \
-        if (mode == 2)                                                                                          \
-            layernorm_rows_kernel<n, 2><<<blocks, 256, 0, ctx.stream>>>(X, Y, rows, rpw, eps, gamma, beta, shift0, \
-                                                                        shift1, scale0, scale1, mod_div, mod_ld); \
-        else                                                                                                    \
-            layernorm_rows_kernel<n, 1><<<blocks, 256, 0, ctx.stream>>>(X, Y, rows, rpw, eps, gamma, beta, shift0, \
-                                                                        shift1, scale0, scale1, mod_div, mod_ld); \
+        const WaitCtl wc{ctx.err, ctx.wait_limit_ns};
+#define WAN_LN_ROWS(n)                                                                                            \
+    case n:                                                                                                       \
+        if (mode == 2)                                                                                            \
+            layernorm_rows_kernel<n, 2><<<blocks, 256, LN_SMEM, ctx.stream>>>(X, Y, rows, rpw, eps, gamma, beta,   \
+                                                                              shift1, scale1, mod_div, mod_ld, wc); \
+        else                                                                                                      \
+            layernorm_rows_kernel<n, 1><<<blocks, 256, LN_SMEM, ctx.stream>>>(X, Y, rows, rpw, eps, gamma, beta,   \
+                                                                              shift1, scale1, mod_div, mod_ld, wc); \
         break;
         switch (D / 256) {
             WAN_LN_ROWS(1) WAN_LN_ROWS(2) WAN_LN_ROWS(3) WAN_LN_ROWS(4) WAN_LN_ROWS(6)

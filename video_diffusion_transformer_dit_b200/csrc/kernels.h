@@ -76,6 +76,7 @@ struct LaunchCtx {
 // Raise the dynamic shared-memory limit of the tcgen05 kernels (once per
 // process and device; call outside stream capture).
 cudaError_t init_kernel_attributes();
+cudaError_t init_layernorm_attributes();  // part of init_kernel_attributes
 
 // Tensor maps (TMA descriptors).
 bool make_tmap_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld_elems,

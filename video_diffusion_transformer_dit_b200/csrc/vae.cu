@@ -229,8 +229,6 @@ int grid_for(long long total, int sms) {
     return (int)g;
 }
 
-size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
 // ------------------------------------------------------------------ decoder description
 enum Kind { K_CONV, K_RES, K_ATTN, K_UP3D, K_UP2D, K_NORM };
 struct Entry {
@@ -723,7 +721,6 @@ wan_status wan_vae_load_weights(wan_vae* v, int n, const char* const* names, con
     wan_status first = WAN_OK;
     void* tmp = nullptr;
     size_t tmp_bytes = 0;
-    LaunchCtx ctx{st, nullptr, 0, v->num_sms, nullptr};
     for (int i = 0; i < n; ++i) {
         if (!names[i] || !ptrs[i]) {
             if (first == WAN_OK) first = vfail(v, WAN_EINVAL, "null name or pointer");
@@ -787,7 +784,6 @@ wan_status wan_vae_load_weights(wan_vae* v, int n, const char* const* names, con
     }
     VCU(cudaStreamSynchronize(st), "weight load");
     if (tmp) cudaFree(tmp);
-    (void)ctx;
     return first;
 }
 
