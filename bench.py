@@ -315,12 +315,12 @@ def run_ours(args, rank, world, local_rank):
         "tc_peak_frac_of": f"{peaks['source']} bf16 {peaks['bf16_tflops']} TFLOP/s (burst)",
         "tc_peak_frac_spec": flops / (ms * 1e-3) / 1e12 / SPEC_BF16_TFLOPS,
         "tc_peak_frac_spec_of": f"dense bf16 spec {SPEC_BF16_TFLOPS} TFLOP/s",
-        "roofline": {"kernel": "self-attention (attn_tc_kernel)", "bound": "tensor", "achieved": achieved,
+        "roofline": {"kernel": "self-attention (attn_pair_kernel)", "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None,
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
                      "flops_per_launch": sa_flops, "avg_launch_ms": sa_avg_ms, "launches_per_step": sa_n,
                      # the committed ncu capture is of the default workload's self-attention launch
-                     "traffic": measured_traffic("attn_tc_kernel",
+                     "traffic": measured_traffic("attn_pair_kernel",
                                                  "video_diffusion_transformer_dit_b200/csrc/attention.cu")
                      if args.workload == DEFAULT_WORKLOAD else None,
                      "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},

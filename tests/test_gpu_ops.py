@@ -244,6 +244,60 @@ def test_attention_large_logits_rescale():
     assert rel_l2(o, ref) < TOL
 
 
+@pytest.mark.parametrize("Lq,Lk", [(1100, 777), (1300, 640), (513, 1000), (2048, 2056)])
+def test_attention_sm_pairs_ragged(Lq, Lk):
+    """Key sets longer than four tiles run on SM pairs (512 queries per cluster,
+    each CTA holding 64-key halves of K and 64-column halves of V).  Lq = 1100
+    leaves the last pair's odd CTA without a valid row, 1300 with some, 513 the
+    even CTA with one; Lk = 777 and 2056 end in a tile whose odd-CTA key half is
+    all padding.  B = 2, 3 heads against the oracle per element."""
+    Bn, heads = 2, 3
+    D = heads * 128
+    g = torch.Generator().manual_seed(Lq + 3 * Lk)
+    q = torch.randn(Bn * Lq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(Bn * Lk, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(Bn * Lk, D, generator=g).to(torch.bfloat16)
+    o = torch.full((Bn * Lq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    B().op_attention(q.cuda(), k.cuda(), v.cuda(), o, Bn, heads, Lq, Lk)
+    B().op_sync()
+    ref = O.attention(q.to(DT).reshape(Bn, Lq, heads, 128), k.to(DT).reshape(Bn, Lk, heads, 128),
+                      v.to(DT).reshape(Bn, Lk, heads, 128)).reshape(Bn * Lq, D)
+    assert not torch.isnan(o.float()).any()
+    assert rel_l2(o, ref) < TOL
+
+
+def test_attention_sm_pairs_zero_wait_limit_reports_and_recovers():
+    """Waits that give up at the first open barrier in both CTAs of every pair:
+    the op reports WAN_ETIMEOUT (or finishes), the pair drains its loads and
+    MMAs, and the next run with the normal limit gives the reference bits."""
+    Bn, heads, L = 1, 4, 2048
+    D = heads * 128
+    g = torch.Generator().manual_seed(5)
+    q, k, v = (torch.randn(Bn * L, D, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    ref = torch.empty(Bn * L, D, dtype=torch.bfloat16, device="cuda")
+    B().op_attention(q, k, v, ref, Bn, heads, L, L)
+    B().op_sync()
+    seen = []
+    B().op_set_wait_limit_ns(0)
+    try:
+        for _ in range(3):
+            o = torch.empty_like(ref)
+            B().op_attention(q, k, v, o, Bn, heads, L, L)
+            try:
+                B().op_sync()
+                seen.append("WAN_OK")
+            except B().WanError as e:
+                seen.append(e.name)
+    finally:
+        B().op_set_wait_limit_ns(2_000_000_000)
+    assert "WAN_ETIMEOUT" in seen, seen
+    assert set(seen) <= {"WAN_ETIMEOUT", "WAN_OK"}, seen
+    again = torch.empty_like(ref)
+    B().op_attention(q, k, v, again, Bn, heads, L, L)
+    B().op_sync()
+    assert torch.equal(again.cpu(), ref.cpu())
+
+
 # ------------------------------------------------------------------ norms
 @pytest.mark.parametrize("D", [1536, 3072, 5120])
 def test_layernorm_modulated(D):

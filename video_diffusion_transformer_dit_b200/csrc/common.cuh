@@ -99,6 +99,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// mbar_wait without suspending: the waiting thread keeps probing (for a
+// single issuing thread whose wake-up latency would sit on the critical path).
+__device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, volatile int* abort, const WaitCtl& wc) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try(bar, parity)) return true;
+        if ((n & 63) == 0) {
+            if (*abort) return false;
+            if (wc.limit_ns == 0 || global_ns() - t0 > wc.limit_ns) {
+                *abort = 1;
+                if (wc.err) atomicExch(wc.err, ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
 // Teardown wait that ignores the abort flag (used to drain own async work).
 __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = global_ns();
@@ -385,6 +403,14 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1)
         : "memory");
 }
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint32_t bar, int c0, int c1,
+                                                 int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
 // Tensor memory of a pair: one warp of each CTA executes alloc / dealloc.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
@@ -433,6 +459,11 @@ __device__ __forceinline__ bool elect_one() {
         "selp.b32 %0, 1, 0, P;\n\t}"
         : "=r"(pred));
     return pred != 0;
+}
+
+// 16-byte store to this CTA's shared memory (shared-space address).
+__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 // Named barrier over `count` threads (a multiple of 32), id 1..15.
