@@ -380,13 +380,16 @@ def test_rmsnorm_rope(rope):
 
 
 # ------------------------------------------------------------------ q/k RMSNorm split across the QKV epilogue
+@pytest.mark.parametrize("grid", [(3, 5, 9), (5, 12, 13)], ids=["L135", "L780"])
 @pytest.mark.parametrize("rope", [True, False])
-def test_qk_norm_epilogue_row_factors_and_attention(rope):
+def test_qk_norm_epilogue_row_factors_and_attention(rope, grid):
     """The self-attention path with RMSNorm across heads in two parts: the QKV
     GEMM epilogue (gain, RoPE, per-head sums of squares), the key row factors in
     place, the query row factors inside the attention -- against the oracle's
-    RMSNorm + RoPE + attention.  B = 2, L = 135 tokens (a ragged second tile)."""
-    Fp, Hp, Wp = 3, 5, 9
+    RMSNorm + RoPE + attention.  B = 2; L = 135 tokens (two key tiles, the
+    single-SM kernel, a ragged second tile) and L = 780 (seven key tiles, the
+    SM-pair kernel: the second pair's odd CTA holds 12 valid query rows)."""
+    Fp, Hp, Wp = grid
     L, Bn, D, h, eps = Fp * Hp * Wp, 2, 1536, 12, 1e-6
     R = Bn * L
     g = torch.Generator().manual_seed(40)
