@@ -87,7 +87,13 @@ WANDIT_API wan_status wan_op_gemm(const void* A, int64_t lda, const void* W, int
  * ("WanTransformerBlock" attn1 / attn2; bidirectional full attention,
  * 【VLA与模仿学习】Wan2.1框架与训练源码导读 §5.2).  Row (b, l) of Q/O starts at
  * q + (b * Lq + l) * ldq; of K/V at k + (b * Lk + l) * ldk; head h occupies
- * columns [128 h, 128 h + 128).  bf16 in/out, fp32 online softmax.          */
+ * columns [128 h, 128 h + 128).  bf16 in/out, fp32 online softmax.  Key
+ * rows past Lk in the last 128-key tile are masked.  Errors, reported before
+ * any launch: WAN_EINVAL for a null pointer; WAN_ESHAPE for B < 0, heads <= 0,
+ * Lq < 0, Lk <= 0, a leading dimension that is not a multiple of 8 elements,
+ * or a pointer that is not 16-byte aligned.  B = 0 or Lq = 0 launches
+ * nothing.  Up to four key tiles (Lk <= 512) run on one SM per CTA; longer
+ * key sets run on SM pairs (clusters of two CTAs).                          */
 WANDIT_API wan_status wan_op_attention(const void* q, int64_t ldq, const void* k, int64_t ldk,
                             const void* v, int64_t ldv, void* o, int64_t ldo,
                             int B, int heads, int Lq, int Lk, void* stream);
@@ -96,7 +102,9 @@ WANDIT_API wan_status wan_op_attention(const void* q, int64_t ldq, const void* k
  * multiplied by its RMSNorm factor rsqrt(sum_{g < ngroups} q_ssq[(b * Lq + l) *
  * ssq_ld + g] / (128 * heads) + eps), the sums of squares coming from the
  * WAN_EPI_QK_NORM epilogue (RMSNorm across heads: "qk_norm =
- * rms_norm_across_heads").  Same layouts and limits as wan_op_attention.     */
+ * rms_norm_across_heads").  Same layouts and limits as wan_op_attention;
+ * also WAN_EINVAL for a null q_ssq and WAN_ESHAPE for ngroups <= 0 or
+ * ssq_ld < ngroups.                                                          */
 WANDIT_API wan_status wan_op_attention_qnorm(const void* q, int64_t ldq, const void* k, int64_t ldk,
                             const void* v, int64_t ldv, void* o, int64_t ldo,
                             int B, int heads, int Lq, int Lk,
