@@ -77,6 +77,22 @@ def test_null_handle_calls_are_refused(lib):
     assert lib.wan_dit_last_error(None) == b"null handle"
 
 
+def test_attention_ops_reject_bad_arguments_before_the_device(lib):
+    """Null pointers give WAN_EINVAL and impossible shapes WAN_ESHAPE, both
+    before the op looks for a device (the checks run here without one)."""
+    fake = ctypes.c_void_p(1 << 20)            # never dereferenced: every call below is refused first
+    att, attq = lib.wan_op_attention, lib.wan_op_attention_qnorm
+    assert att(None, 128, fake, 128, fake, 128, fake, 128, 1, 1, 128, 128, None) == 1
+    assert att(fake, 128, fake, 128, fake, 128, None, 128, 1, 1, 128, 128, None) == 1
+    for B, heads, Lq, Lk in ((-1, 1, 128, 128), (1, 0, 128, 128), (1, 1, -1, 128), (1, 1, 128, 0)):
+        assert att(fake, 128, fake, 128, fake, 128, fake, 128, B, heads, Lq, Lk, None) == 2
+    assert attq(fake, 128, fake, 128, fake, 128, fake, 128, 1, 1, 128, 128, None, 1, 1,
+                ctypes.c_float(1e-6), None) == 1
+    for ssq_ld, ngroups in ((1, 0), (1, 2)):
+        assert attq(fake, 128, fake, 128, fake, 128, fake, 128, 1, 1, 128, 128, fake, ssq_ld, ngroups,
+                    ctypes.c_float(1e-6), None) == 2
+
+
 def test_flow_sigmas_match_oracle(lib):
     """The host-side sigma schedule against the oracle's reading R22."""
     import torch

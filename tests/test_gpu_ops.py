@@ -266,6 +266,30 @@ def test_attention_sm_pairs_ragged(Lq, Lk):
     assert rel_l2(o, ref) < TOL
 
 
+@pytest.mark.parametrize("Lk", [226, 1024])
+def test_attention_rejects_misaligned_operands_before_launch(Lk):
+    """A pointer off the 16-byte grid or a leading dimension that is not a
+    multiple of 8 elements is WAN_ESHAPE, for the single-SM (226 keys) and the
+    SM-pair (1024 keys) kernels alike, and nothing is written."""
+    Bn, heads, Lq = 1, 2, 300
+    D = heads * 128
+    q = torch.randn(Bn * Lq + 1, D + 8).to(torch.bfloat16).cuda()
+    kv = torch.randn(Bn * Lk + 1, D + 8).to(torch.bfloat16).cuda()
+    o = torch.full((Bn * Lq + 1, D + 8), 7.0, dtype=torch.bfloat16, device="cuda")
+    qp, kp, op = q.data_ptr(), kv.data_ptr(), o.data_ptr()
+    ld = D + 8
+    bad = [(qp + 2, ld, kp, ld, op, ld),          # q not 16-byte aligned
+           (qp, ld, kp, ld, op + 2, ld),          # o not 16-byte aligned
+           (qp, ld - 1, kp, ld, op, ld),          # ldq not a multiple of 8
+           (qp, ld, kp, ld - 4, op, ld)]          # ldk not a multiple of 8
+    for q_, ldq, k_, ldk, o_, ldo in bad:
+        with pytest.raises(B().WanError) as e:
+            B().op_attention_ptr(q_, ldq, k_, ldk, k_, ldk, o_, ldo, Bn, heads, Lq, Lk)
+        assert e.value.name == "WAN_ESHAPE"
+    B().op_sync()
+    assert torch.all(o.cpu() == 7.0)
+
+
 def test_attention_sm_pairs_zero_wait_limit_reports_and_recovers():
     """Waits that give up at the first open barrier in both CTAs of every pair:
     the op reports WAN_ETIMEOUT (or finishes), the pair drains its loads and
