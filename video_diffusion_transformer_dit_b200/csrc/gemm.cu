@@ -312,9 +312,30 @@ __device__ __forceinline__ void qk_position(const EpiParams& e, int row, int& f,
     jj = rem - ii * e.rope.Wp;
 }
 
+// RoPE (cos, sin) of the 16 rotation pairs of chunk K (32 columns) of a head,
+// for the 22 / 21 / 21 pairs per axis of a 44 / 42 / 42 split: every pair's
+// axis is fixed by the chunk, one multiply-add per table address.
+template <int K>
+__device__ __forceinline__ void qk_rope_load_fixed(const RopeTables& rt, int f, int ii, int jj, float2 (&cs)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int q = 16 * K + i;
+        const float2* a = q < 22 ? rt.t + q * rt.Fp + f : (q < 43 ? rt.h + (q - 22) * rt.Hp + ii : rt.w + (q - 43) * rt.Wp + jj);
+        cs[i] = __ldg(a);
+    }
+}
+
 // RoPE (cos, sin) of the 16 rotation pairs of a 32-column chunk at token
 // position (f, ii, jj), from the pair-major tables; loaded ahead of the chunk.
 __device__ __forceinline__ void qk_rope_load(const EpiParams& e, int c, int f, int ii, int jj, float2 (&cs)[16]) {
+    if (e.rope.nt == 22 && e.rope.nh == 21 && e.rope.nw == 21) {
+        switch ((c & 127) >> 5) {
+            case 0: qk_rope_load_fixed<0>(e.rope, f, ii, jj, cs); return;
+            case 1: qk_rope_load_fixed<1>(e.rope, f, ii, jj, cs); return;
+            case 2: qk_rope_load_fixed<2>(e.rope, f, ii, jj, cs); return;
+            default: qk_rope_load_fixed<3>(e.rope, f, ii, jj, cs); return;
+        }
+    }
     const int p0 = (c & 127) >> 1;
 #pragma unroll
     for (int i = 0; i < 16; ++i) cs[i] = __ldg(rope_entry_pm(e.rope, p0 + i, f, ii, jj));
