@@ -27,6 +27,11 @@ WORKLOADS = {
     # one block + head, 192 tokens: the case the oracle finishes in seconds
     "wan1.3b-1blk-3x16x16": dict(model="wan2.1-1.3b", overrides=dict(num_blocks=1),
                                  latent=(1, 16, 3, 16, 16), text_len=32, timesteps=(500.0,)),
+    # one block + head on a CFG pair, 720 tokens: self-attention and the block GEMMs on SM pairs
+    # (the second 512-query pair ragged), still a case the oracle finishes in seconds
+    "wan1.3b-1blk-5x24x24-cfg2": dict(model="wan2.1-1.3b", overrides=dict(num_blocks=1),
+                                      latent=(2, 16, 5, 24, 24), text_len=32, timesteps=(500.0,),
+                                      same_latent=True),
     # 33 frames 352x640 -> 7920 tokens, 30 blocks
     "wan1.3b-33f-352x640": dict(model="wan2.1-1.3b", overrides={},
                                 latent=(1, 16, 9, 44, 80), text_len=226, timesteps=(999.0,)),
